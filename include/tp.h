@@ -1,0 +1,219 @@
+/*
+ * tp.h -- C ABI of libtp: the Megatron-style tensor-parallel MLP over t virtual shards held in one
+ * GPU's memory, ring-order collectives over those shards, and the four sharded-matmul cases.
+ *
+ * Sources (pages cited by title and section):
+ *   [TPSP] "张量并行与序列并行" (hs-black.github.io, scaling-tensor-parallel)
+ *   [CH06] "Scaling Book 入门第 6 章：分片矩阵乘法 — 分布式计算的核心" (r00kie-liu.github.io, scaling-infra-ch06)
+ *   [CH05] "Scaling Book 入门第 5 章：Sharded Matrices 上篇 — 集合通信原语" (r00kie-liu.github.io, scaling-infra-ch05)
+ *   [PFY]  pufanyi.com "ml-revisit-infra", section "Tensor Parallel"
+ *
+ * Conventions shared by every entry point
+ *   - All matrices are row-major. Weights are [in, out] (a linear layer is Y = X W, W of shape [k, n]).
+ *   - "bf16" buffers are uint16_t bit patterns of bfloat16; "f32" buffers are IEEE binary32.
+ *   - Every data pointer is a DEVICE pointer, except arrays of shard pointers ("const T* const* p"),
+ *     which are HOST arrays of t device pointers. t (the TP degree) is 1..TP_MAX_SHARDS.
+ *   - The caller allocates and frees every buffer. The library allocates no device memory; it keeps
+ *     one device status word and the code it needs.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream). Every call is asynchronous on it.
+ *     Argument errors are returned before anything is launched; a failed launch returns TP_ECUDA.
+ *     tp_last_error() gives a one-line message for the last failure on the calling host thread.
+ *   - Device pointers must be 16-byte aligned and row strides a multiple of 16 bytes (8 bf16 or 4 f32
+ *     elements) where a function says "aligned"; otherwise TP_EALIGN. A dimension that t must divide
+ *     and does not gives TP_EDIVIS (nothing is padded).
+ *   - Buffers must not overlap unless a function states otherwise.
+ *   - Device-side waits are bounded; a wait that runs out records TP_ETIMEOUT in the device status
+ *     word (read it with tp_device_status) and the kernel returns without finishing its work.
+ */
+#ifndef TP_H_
+#define TP_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define TP_MAX_SHARDS 16
+
+typedef enum {
+  TP_OK = 0,
+  TP_EINVAL = 1,        /* null pointer, non-positive size, bad enum value */
+  TP_ESHAPE = 2,        /* sizes inconsistent with each other */
+  TP_EDIVIS = 3,        /* t does not divide a dimension it must split */
+  TP_EALIGN = 4,        /* pointer or row stride not 16-byte aligned */
+  TP_ECUDA = 5,         /* a CUDA runtime/driver call failed */
+  TP_ETIMEOUT = 6,      /* a bounded device-side wait ran out (reported by tp_device_status) */
+  TP_EUNSUPPORTED = 7,  /* valid request this build does not implement */
+  TP_ENOSPACE = 8       /* a caller-supplied workspace is too small */
+} tp_status;
+
+typedef enum { TP_F32 = 0, TP_BF16 = 1 } tp_dtype;
+
+/* Activation applied in the column-parallel GEMM's epilogue. It is element-wise, so each shard
+ * applies it to its own columns ([TPSP] §MLP：先列后行，只通信一次). GELU is the exact erf form.
+ * SWIGLU reads a fused [gate | up] operand and writes SiLU(gate) * up (one output per pair). */
+typedef enum { TP_ACT_NONE = 0, TP_ACT_GELU = 1, TP_ACT_GELU_TANH = 2, TP_ACT_SWIGLU = 3 } tp_act;
+
+/* What tp_mlp_fwd returns after the row-parallel GEMM. */
+typedef enum {
+  TP_OUT_PARTIALS = 0,  /* the t unreduced partial sums {U} ([TPSP] §矩阵乘法的两种切法, row-parallel) */
+  TP_OUT_RS = 1,        /* ReduceScatter along tokens: shard r gets rows [rN/t,(r+1)N/t) of sum U */
+  TP_OUT_AR = 2,        /* AllReduce in one pass: every shard gets sum U */
+  TP_OUT_RS_AG = 3      /* AllReduce as ReduceScatter along tokens then AllGather (bit-identical to AR) */
+} tp_reduce;
+
+/* Strategies of tp_sharded_matmul ([CH06] §6.2, four cases of C[B,F] = X[B,D] W[D,F]). */
+typedef enum {
+  TP_CASE1_LOCAL = 0,
+  TP_CASE2_ALLGATHER = 0, TP_CASE2_ALLREDUCE = 1,
+  TP_CASE3_ALLREDUCE = 0, TP_CASE3_RS_B = 1, TP_CASE3_RS_F = 2,
+  TP_CASE4_GATHER_X = 0, TP_CASE4_GATHER_W = 1
+} tp_strategy;
+
+/* ------------------------------------------------------------------------------------------------
+ * Status and diagnostics
+ * ------------------------------------------------------------------------------------------------ */
+const char* tp_status_str(tp_status s);
+/* One-line description of the last failure returned on the calling host thread ("" if none). */
+const char* tp_last_error(void);
+/* Synchronises the current device, then returns TP_ETIMEOUT if any kernel recorded a wait that ran
+ * out since the last clear (TP_OK otherwise, TP_ECUDA if synchronising failed). clear != 0 resets
+ * the word. *where (optional, host) receives the code of the wait that ran out. */
+tp_status tp_device_status(int clear, uint32_t* where);
+/* Budget, in SM clock cycles, of every bounded device-side wait issued by later launches
+ * (0 restores the default of about two seconds). */
+void tp_set_wait_budget(uint64_t cycles);
+/* Launches one kernel that waits, bounded by `budget_cycles`, on a device flag that nothing sets,
+ * so that the wait runs out and records TP_ETIMEOUT in the status word (failure-path self test). */
+tp_status tp_selftest_wait_timeout(uint64_t budget_cycles, void* stream);
+/* Number of streaming multiprocessors of the current device (grid sizing), or -1 on error. */
+int tp_num_sms(void);
+
+/* ------------------------------------------------------------------------------------------------
+ * Weight shard layouts (bit copies). Outputs are stacked: shard r starts at out + r * (shard size).
+ * All aligned (inputs' row strides ld_* in elements). One-off conversions, not on the hot loop.
+ * ------------------------------------------------------------------------------------------------ */
+/* Column-parallel split of W[K, N] (row stride ld): out[r] = W[:, rN/t:(r+1)N/t], shape [K, N/t].
+ * ([TPSP] §矩阵乘法的两种切法, first identity; [CH06] §6.7 Column Parallel Linear.) */
+tp_status tp_shard_cols(const uint16_t* w, int64_t ld, int64_t K, int64_t N, int t, uint16_t* out, void* stream);
+/* Row-parallel split of W[K, N] (row stride ld): out[r] = W[rK/t:(r+1)K/t, :], shape [K/t, N].
+ * ([TPSP] §矩阵乘法的两种切法, second identity; [CH06] §6.7 Row Parallel Linear.) */
+tp_status tp_shard_rows(const uint16_t* w, int64_t ld, int64_t K, int64_t N, int t, uint16_t* out, void* stream);
+/* Fused SwiGLU gate|up layout of W_gate[h, F] and W_up[h, F] (row strides ld_g, ld_u):
+ * out[r] = [W_gate[:, F-range r] | W_up[:, F-range r]], shape [h, 2F/t] -- a rank's gate and up
+ * columns cover the same F indices ([TPSP] §MLP, SwiGLU paragraph). Gate first, then up. */
+tp_status tp_shard_gate_up(const uint16_t* w_gate, int64_t ld_g, const uint16_t* w_up, int64_t ld_u,
+                           int64_t h, int64_t F, int t, uint16_t* out, void* stream);
+/* Rank-grouped fused QKV layout ([TPSP] §注意力：按头切 fused-QKV bullet, §GQA). W_q[h, n_h*d_h],
+ * W_k/W_v[h, n_kv*d_h] (row strides ld_q, ld_k, ld_v). out[r] = [Q heads of rank r | its K heads | its
+ * V heads], heads ascending, d_h columns each; shape [h, (n_h/t + 2*kv)*d_h] with kv = n_kv/t when
+ * t <= n_kv, else kv = 1 and rank r takes KV head floor(r*n_kv/t) (replication for n_kv < t <= n_h).
+ * t must divide n_h, n_kv must divide n_h, and t | n_kv or n_kv | t (TP_EDIVIS otherwise). */
+tp_status tp_shard_qkv(const uint16_t* w_q, int64_t ld_q, const uint16_t* w_k, int64_t ld_k,
+                       const uint16_t* w_v, int64_t ld_v, int64_t h, int n_h, int n_kv, int d_h, int t,
+                       uint16_t* out, void* stream);
+
+/* ------------------------------------------------------------------------------------------------
+ * Ring collectives over t shard buffers resident in this GPU's memory ([CH05] §5.2 环形算法, §5.3;
+ * [CH06] §6.4). `in` and `out` are host arrays of t device pointers; buffers are contiguous
+ * [rows, cols] matrices of `dtype`.
+ *
+ * Summation order (the pages fix the ring, device i passing to i+1 and accumulating at every step,
+ * and that device r ends with chunk r; the order of the adds follows from that): chunk c is
+ * (((U[c+1] + U[c+2]) + U[c+3]) + ... ) + U[c], indices mod t, one binary32 add at a time. bf16 inputs
+ * are widened to binary32, summed in that order and rounded once to bf16 (nearest-even).
+ * Chunk r is the row block [r*rows/t, (r+1)*rows/t) (axis 0) or column block (axis 1).
+ * Results are bit-exact and independent of launch shape; no atomics are used.
+ * ------------------------------------------------------------------------------------------------ */
+/* ReduceScatter: in[s] is [rows, cols]; out[r] receives chunk r of the sum: [rows/t, cols] (axis 0)
+ * or [rows, cols/t] (axis 1). */
+tp_status tp_reduce_scatter(const void* const* in, void* const* out, int64_t rows, int64_t cols, int axis,
+                            tp_dtype dtype, int t, void* stream);
+/* AllGather: in[r] is shard r of the gathered [rows, cols] matrix ([rows/t, cols] for axis 0,
+ * [rows, cols/t] for axis 1); every out[s] receives the whole [rows, cols] in shard order. In-place is
+ * allowed for axis 0 when in[r] == out[r] + r*(rows/t)*cols (each shard's piece already in place). */
+tp_status tp_all_gather(const void* const* in, void* const* out, int64_t rows, int64_t cols, int axis,
+                        tp_dtype dtype, int t, void* stream);
+/* AllReduce (= ReduceScatter + AllGather, done in one pass): every out[s] receives the ring-ordered
+ * sum of the t in[] buffers; all replicas are bit-identical. in[s] == out[s] (in place) is allowed. */
+tp_status tp_all_reduce(const void* const* in, void* const* out, int64_t rows, int64_t cols,
+                        tp_dtype dtype, int t, void* stream);
+
+/* ------------------------------------------------------------------------------------------------
+ * GEMMs on the tensor cores (bf16 inputs, fp32 accumulation)
+ * ------------------------------------------------------------------------------------------------ */
+/* Grouped GEMM: for g < groups, c[g] = act(a[g] . b[g]) with a[g] [M, K] bf16, b[g] [K, Nb] bf16
+ * (Nb = N, or 2N for TP_ACT_SWIGLU where b[g] = [gate | up]) and c[g] [M, N] of c_dtype
+ * (TP_ACT_NONE may write f32 or bf16; the activations write bf16). a[] entries may repeat (a shared
+ * input). Aligned; K and N must be multiples of 8. groups <= TP_MAX_SHARDS. */
+tp_status tp_grouped_gemm(int groups, const uint16_t* const* a, const uint16_t* const* b, void* const* c,
+                          int64_t M, int64_t N, int64_t K, tp_act act, tp_dtype c_dtype, void* stream);
+/* Column-parallel linear ([TPSP] §矩阵乘法的两种切法; [CH06] §6.7): y[r] = act(x . w[r]) for every
+ * shard r, from the full x [N, k] (shared by all shards) and the stacked shards w [t][k][n/t]
+ * ([t][k][2n/t] = [gate_r | up_r] for SWIGLU, as written by tp_shard_gate_up). y is stacked
+ * [t][N][n/t] bf16. No communication. */
+tp_status tp_column_linear(const uint16_t* x, int64_t N, int64_t k, int64_t n, int t, tp_act act,
+                           const uint16_t* w, uint16_t* y, void* stream);
+/* Row-parallel linear: partials[r] = x[r] . w[r], fp32 [N, n], from stacked x [t][N][k/t] and
+ * w [t][k/t][n]. The true output is sum_r partials[r] (a following AllReduce or ReduceScatter). */
+tp_status tp_row_linear(const uint16_t* x, int64_t N, int64_t k, int64_t n, int t, const uint16_t* w,
+                        float* const* partials, void* stream);
+
+/* ------------------------------------------------------------------------------------------------
+ * The tensor-parallel MLP forward ([TPSP] §MLP：先列后行，只通信一次; [PFY] §Tensor Parallel;
+ * [CH06] §6.9 Problem 5): Z_r = act(X W_in[r]) (column-parallel, local), U_r = Z_r W_down[r]
+ * (row-parallel, full-shape partial), then the collective `mode` selects.
+ *   x       bf16 [N, h], shared by all shards
+ *   w_in    bf16 stacked [t][h][F/t] (GELU/NONE) or [t][h][2F/t] (SWIGLU, from tp_shard_gate_up)
+ *   w_down  bf16 stacked [t][F/t][h] (from tp_shard_rows)
+ *   z_ws    bf16 workspace [t][N][F/t] (the activations Z_r)
+ *   partials t fp32 [N, h] buffers (the {U}); required for every mode
+ *   out     t fp32 buffers: unused for PARTIALS; [N/t, h] for RS (t | N); [N, h] for AR and RS_AG
+ * Aligned; h and F/t multiples of 8. */
+tp_status tp_mlp_fwd(const uint16_t* x, int64_t N, int64_t h, int64_t F, int t, tp_act act,
+                     const uint16_t* w_in, const uint16_t* w_down, uint16_t* z_ws, float* const* partials,
+                     tp_reduce mode, float* const* out, void* stream);
+
+/* ------------------------------------------------------------------------------------------------
+ * The four sharded-matmul cases of C[B,F] = X[B,D] . W[D,F] over t shards ([CH06] §6.2, §6.9
+ * Problems 4 and 9). x[] and w[] are host arrays of t device pointers (bf16, row-major); entries of a
+ * replicated operand may point to the same buffer. c[] receives t outputs of c_dtype.
+ *   case 1 X[B_X, D] . W[D, F]: x[i] [B/t, D], w[i] [D, F] -> c[i] [B/t, F]; no communication.
+ *   case 2 X[B, D_X] . W[D, F]: x[i] [B, D/t], w[i] [D, F] (replicated)
+ *       ALLGATHER: every shard gathers X and computes the full C -> c[i] [B, F] (t x the FLOPs)
+ *       ALLREDUCE: shard i multiplies by its row block of W, then AllReduce -> c[i] [B, F]
+ *   case 3 X[B, D_X] . W[D_X, F]: x[i] [B, D/t], w[i] [D/t, F] -> partial C{U_X}, then
+ *       ALLREDUCE -> c[i] [B, F]; RS_B -> c[i] [B/t, F]; RS_F -> c[i] [B, F/t]
+ *   case 4 X[B_X, D] . W[D, F_X] (only diagonal blocks as is), fixed by
+ *       GATHER_X -> c[i] [B, F/t]; GATHER_W -> c[i] [B/t, F]
+ * Partial sums are fp32 and reduced in the ring order above; a bf16 c_dtype rounds once at the end.
+ * The workspace (device, >= tp_sharded_matmul_ws_bytes) holds gathered operands or partials. */
+size_t tp_sharded_matmul_ws_bytes(int case_id, int strategy, int64_t B, int64_t D, int64_t F, int t);
+tp_status tp_sharded_matmul(int case_id, int strategy, const uint16_t* const* x, const uint16_t* const* w,
+                            int64_t B, int64_t D, int64_t F, int t, void* const* c, tp_dtype c_dtype,
+                            void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------------------------------
+ * One tensor-parallel transformer layer without its attention core ([TPSP] §注意力：按头切 and §MLP;
+ * 2 AllReduces per layer forward): qkv[r] = X W_qkv[r] (column-parallel; its output feeds the
+ * attention core, which is outside this library); attn = AllReduce_r(O[r] W_o[r]); h1 = X + attn (fp32);
+ * the MLP (SwiGLU) runs on bf16(h1); y = h1 + AllReduce_r(MLP partials).
+ *   x      bf16 [N, h];  o: t device pointers, bf16 [N, n_h*d_h/t] (each shard's attention output)
+ *   w_qkv  bf16 stacked [t][h][(n_h/t + 2kv)*d_h] (tp_shard_qkv); w_o bf16 stacked [t][n_h*d_h/t][h]
+ *   w_gu   bf16 stacked [t][h][2F/t];  w_down bf16 stacked [t][F/t][h]
+ *   qkv_out bf16 stacked [t][N][(n_h/t + 2kv)*d_h]
+ *   h1     t fp32 [N, h] (replicas of the residual stream after attention); h1_bf16 bf16 [N, h]
+ *   z_ws   bf16 [t][N][F/t]; partials t fp32 [N, h]; y t fp32 [N, h]
+ * ------------------------------------------------------------------------------------------------ */
+tp_status tp_layer_fwd(const uint16_t* x, const uint16_t* const* o, int64_t N, int64_t h, int n_h, int n_kv,
+                       int d_h, int64_t F, int t, const uint16_t* w_qkv, const uint16_t* w_o,
+                       const uint16_t* w_gu, const uint16_t* w_down, uint16_t* qkv_out, float* const* h1,
+                       uint16_t* h1_bf16, uint16_t* z_ws, float* const* partials, float* const* y, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TP_H_ */

@@ -1,4 +1,4 @@
-"""Weight shard layouts, written as plain index copies from their definitions (test infrastructure).
+"""Weight shard layouts, written as plain block copies from their definitions (test infrastructure).
 
 All weights are [in, out] row-major, as the pages write a linear layer Y = X W with W of shape [k, n]
 ("张量并行与序列并行", §矩阵乘法的两种切法). Arrays may be any dtype (bf16 bits as uint16 compare byte
@@ -19,8 +19,7 @@ def shard_cols(W: np.ndarray, t: int) -> np.ndarray:
     w = n // t
     out = np.empty((t, k, w), dtype=W.dtype)
     for r in range(t):
-        for j in range(w):
-            out[r, :, j] = W[:, r * w + j]
+        out[r] = W[:, r * w:(r + 1) * w]
     return out
 
 
@@ -34,8 +33,7 @@ def shard_rows(W: np.ndarray, t: int) -> np.ndarray:
     h = k // t
     out = np.empty((t, h, n), dtype=W.dtype)
     for r in range(t):
-        for i in range(h):
-            out[r, i, :] = W[r * h + i, :]
+        out[r] = W[r * h:(r + 1) * h, :]
     return out
 
 
@@ -50,9 +48,8 @@ def shard_gate_up(W_gate: np.ndarray, W_up: np.ndarray, t: int) -> np.ndarray:
     f = F // t
     out = np.empty((t, h, 2 * f), dtype=W_gate.dtype)
     for r in range(t):
-        for j in range(f):
-            out[r, :, j] = W_gate[:, r * f + j]
-            out[r, :, f + j] = W_up[:, r * f + j]
+        out[r, :, :f] = W_gate[:, r * f:(r + 1) * f]
+        out[r, :, f:] = W_up[:, r * f:(r + 1) * f]
     return out
 
 

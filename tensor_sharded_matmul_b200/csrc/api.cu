@@ -1,0 +1,283 @@
+// C entry points that compose the GEMM and ring kernels: the column/row parallel linear layers,
+// the tensor-parallel MLP, the four sharded-matmul cases and one tensor-parallel layer.
+// Argument validation happens here, before anything is launched.
+#include <cstring>
+
+#include "common.cuh"
+
+namespace tpx {
+namespace {
+
+bool valid_act(tp_act a) { return a == TP_ACT_NONE || a == TP_ACT_GELU || a == TP_ACT_GELU_TANH || a == TP_ACT_SWIGLU; }
+bool valid_dtype(tp_dtype d) { return d == TP_F32 || d == TP_BF16; }
+
+EpiKind epi_for(tp_act act, tp_dtype c_dtype) {
+  switch (act) {
+    case TP_ACT_GELU: return EPI_GELU;
+    case TP_ACT_GELU_TANH: return EPI_GELU_TANH;
+    case TP_ACT_SWIGLU: return EPI_SWIGLU;
+    default: return c_dtype == TP_F32 ? EPI_F32 : EPI_BF16;
+  }
+}
+
+GemmArgs gemm_args(int groups, int64_t M, int64_t N, int64_t K, int64_t lda, int64_t ldb, EpiKind epi) {
+  GemmArgs g;
+  std::memset(&g, 0, sizeof(g));
+  g.groups = groups; g.M = M; g.N = N; g.K = K; g.lda = lda; g.ldb = ldb; g.epi = epi;
+  return g;
+}
+
+RingArgs ring_args(RingOp op, int t, int64_t rows, int64_t cols, int axis, tp_dtype din, tp_dtype dout) {
+  RingArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.op = op; a.t = t; a.rows = rows; a.cols = cols; a.axis = axis; a.in_dtype = din; a.out_dtype = dout;
+  a.resid_dtype = TP_F32;
+  return a;
+}
+
+size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
+
+tp_status column_gemm(const uint16_t* x, int64_t N, int64_t k, int64_t n_shard, int t, tp_act act, const uint16_t* w,
+                      uint16_t* y, cudaStream_t s) {
+  const int64_t wn = act == TP_ACT_SWIGLU ? 2 * n_shard : n_shard;
+  GemmArgs g = gemm_args(t, N, n_shard, k, k, wn, epi_for(act, TP_BF16));
+  for (int r = 0; r < t; ++r) {
+    g.a[r] = x;
+    g.b[r] = w + r * k * wn;
+    g.c[r] = y + r * N * n_shard;
+  }
+  return grouped_gemm(g, s);
+}
+
+tp_status row_gemm(const uint16_t* x, int64_t N, int64_t k_shard, int64_t n, int t, const uint16_t* w,
+                   float* const* partials, cudaStream_t s) {
+  GemmArgs g = gemm_args(t, N, n, k_shard, k_shard, n, EPI_F32);
+  for (int r = 0; r < t; ++r) {
+    if (partials[r] == nullptr) return fail(TP_EINVAL, "null partial buffer %d", r);
+    g.a[r] = x + r * N * k_shard;
+    g.b[r] = w + r * k_shard * n;
+    g.c[r] = partials[r];
+  }
+  return grouped_gemm(g, s);
+}
+
+// Reduce the t fp32 partials [N, h] according to `mode` into out.
+tp_status reduce_partials(float* const* partials, int64_t N, int64_t h, int t, tp_reduce mode, float* const* out,
+                          const void* resid, tp_dtype resid_dtype, uint16_t* copy_bf16, cudaStream_t s) {
+  if (mode == TP_OUT_PARTIALS) return TP_OK;
+  if (out == nullptr) return fail(TP_EINVAL, "null output array");
+  for (int r = 0; r < t; ++r)
+    if (out[r] == nullptr) return fail(TP_EINVAL, "null output buffer %d", r);
+  if (mode == TP_OUT_RS) {
+    RingArgs a = ring_args(RING_RS, t, N, h, 0, TP_F32, TP_F32);
+    for (int r = 0; r < t; ++r) { a.in[r] = partials[r]; a.out[r] = out[r]; }
+    return ring_collective(a, s);
+  }
+  if (mode == TP_OUT_AR) {
+    RingArgs a = ring_args(RING_AR, t, N, h, 0, TP_F32, TP_F32);
+    for (int r = 0; r < t; ++r) { a.in[r] = partials[r]; a.out[r] = out[r]; }
+    a.resid = resid; a.resid_dtype = resid_dtype; a.copy_bf16 = copy_bf16;
+    return ring_collective(a, s);
+  }
+  if (mode == TP_OUT_RS_AG) {
+    // ReduceScatter along tokens straight into each shard's own row block of its output, then an
+    // in-place AllGather fills in the other shards' blocks.
+    const int64_t chunk = (N / t) * h;
+    RingArgs rs = ring_args(RING_RS, t, N, h, 0, TP_F32, TP_F32);
+    for (int r = 0; r < t; ++r) { rs.in[r] = partials[r]; rs.out[r] = out[r] + r * chunk; }
+    if (tp_status st = ring_collective(rs, s)) return st;
+    RingArgs ag = ring_args(RING_AG, t, N, h, 0, TP_F32, TP_F32);
+    for (int r = 0; r < t; ++r) { ag.in[r] = out[r] + r * chunk; ag.out[r] = out[r]; }
+    return ring_collective(ag, s);
+  }
+  return fail(TP_EINVAL, "bad reduce mode %d", static_cast<int>(mode));
+}
+
+}  // namespace
+}  // namespace tpx
+
+using namespace tpx;
+
+extern "C" {
+
+tp_status tp_grouped_gemm(int groups, const uint16_t* const* a, const uint16_t* const* b, void* const* c, int64_t M,
+                          int64_t N, int64_t K, tp_act act, tp_dtype c_dtype, void* stream) {
+  if (a == nullptr || b == nullptr || c == nullptr) return fail(TP_EINVAL, "null pointer array");
+  if (groups < 1 || groups > TP_MAX_SHARDS) return fail(TP_EINVAL, "groups=%d outside 1..%d", groups, TP_MAX_SHARDS);
+  if (!valid_act(act) || !valid_dtype(c_dtype)) return fail(TP_EINVAL, "bad activation or dtype");
+  if (act != TP_ACT_NONE && c_dtype != TP_BF16) return fail(TP_EINVAL, "activations write bf16");
+  GemmArgs g = gemm_args(groups, M, N, K, K, act == TP_ACT_SWIGLU ? 2 * N : N, epi_for(act, c_dtype));
+  for (int i = 0; i < groups; ++i) { g.a[i] = a[i]; g.b[i] = b[i]; g.c[i] = c[i]; }
+  return grouped_gemm(g, static_cast<cudaStream_t>(stream));
+}
+
+tp_status tp_column_linear(const uint16_t* x, int64_t N, int64_t k, int64_t n, int t, tp_act act, const uint16_t* w,
+                           uint16_t* y, void* stream) {
+  if (!valid_t(t)) return fail(TP_EINVAL, "t=%d outside 1..%d", t, TP_MAX_SHARDS);
+  if (x == nullptr || w == nullptr || y == nullptr) return fail(TP_EINVAL, "null pointer");
+  if (!valid_act(act)) return fail(TP_EINVAL, "bad activation");
+  if (N <= 0 || k <= 0 || n <= 0) return fail(TP_EINVAL, "non-positive size");
+  if (n % t) return fail(TP_EDIVIS, "t=%d does not divide n=%lld", t, (long long)n);
+  return column_gemm(x, N, k, n / t, t, act, w, y, static_cast<cudaStream_t>(stream));
+}
+
+tp_status tp_row_linear(const uint16_t* x, int64_t N, int64_t k, int64_t n, int t, const uint16_t* w,
+                        float* const* partials, void* stream) {
+  if (!valid_t(t)) return fail(TP_EINVAL, "t=%d outside 1..%d", t, TP_MAX_SHARDS);
+  if (x == nullptr || w == nullptr || partials == nullptr) return fail(TP_EINVAL, "null pointer");
+  if (N <= 0 || k <= 0 || n <= 0) return fail(TP_EINVAL, "non-positive size");
+  if (k % t) return fail(TP_EDIVIS, "t=%d does not divide k=%lld", t, (long long)k);
+  return row_gemm(x, N, k / t, n, t, w, partials, static_cast<cudaStream_t>(stream));
+}
+
+tp_status tp_mlp_fwd(const uint16_t* x, int64_t N, int64_t h, int64_t F, int t, tp_act act, const uint16_t* w_in,
+                     const uint16_t* w_down, uint16_t* z_ws, float* const* partials, tp_reduce mode, float* const* out,
+                     void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (!valid_t(t)) return fail(TP_EINVAL, "t=%d outside 1..%d", t, TP_MAX_SHARDS);
+  if (x == nullptr || w_in == nullptr || w_down == nullptr || z_ws == nullptr || partials == nullptr)
+    return fail(TP_EINVAL, "null pointer");
+  if (!valid_act(act)) return fail(TP_EINVAL, "bad activation");
+  if (mode < TP_OUT_PARTIALS || mode > TP_OUT_RS_AG) return fail(TP_EINVAL, "bad reduce mode");
+  if (N <= 0 || h <= 0 || F <= 0) return fail(TP_EINVAL, "non-positive size");
+  if (F % t) return fail(TP_EDIVIS, "t=%d does not divide F=%lld", t, (long long)F);
+  if (mode != TP_OUT_PARTIALS && N % t) return fail(TP_EDIVIS, "t=%d does not divide the token count %lld", t, (long long)N);
+  const int64_t f = F / t;
+  if (tp_status st = column_gemm(x, N, h, f, t, act, w_in, z_ws, s)) return st;          // Z_r = act(X W_in[r])
+  if (tp_status st = row_gemm(z_ws, N, f, h, t, w_down, partials, s)) return st;         // U_r = Z_r W_down[r]
+  return reduce_partials(partials, N, h, t, mode, out, nullptr, TP_F32, nullptr, s);     // g: the collective
+}
+
+size_t tp_sharded_matmul_ws_bytes(int case_id, int strategy, int64_t B, int64_t D, int64_t F, int t) {
+  if (t < 1 || B <= 0 || D <= 0 || F <= 0) return 0;
+  const size_t T = static_cast<size_t>(t);
+  switch (case_id) {
+    case 2: return strategy == TP_CASE2_ALLGATHER ? T * align256(size_t(B) * D * 2) : T * align256(size_t(B) * F * 4);
+    case 3: return T * align256(size_t(B) * F * 4);
+    case 4: return strategy == TP_CASE4_GATHER_X ? T * align256(size_t(B) * D * 2) : T * align256(size_t(D) * F * 2);
+    default: return 0;
+  }
+}
+
+tp_status tp_sharded_matmul(int case_id, int strategy, const uint16_t* const* x, const uint16_t* const* w, int64_t B,
+                            int64_t D, int64_t F, int t, void* const* c, tp_dtype c_dtype, void* ws, size_t ws_bytes,
+                            void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (!valid_t(t)) return fail(TP_EINVAL, "t=%d outside 1..%d", t, TP_MAX_SHARDS);
+  if (x == nullptr || w == nullptr || c == nullptr) return fail(TP_EINVAL, "null pointer array");
+  if (!valid_dtype(c_dtype)) return fail(TP_EINVAL, "bad dtype");
+  if (B <= 0 || D <= 0 || F <= 0) return fail(TP_EINVAL, "non-positive size");
+  for (int i = 0; i < t; ++i)
+    if (x[i] == nullptr || w[i] == nullptr || c[i] == nullptr) return fail(TP_EINVAL, "null shard pointer %d", i);
+  const size_t need = tp_sharded_matmul_ws_bytes(case_id, strategy, B, D, F, t);
+  if (need > 0 && (ws == nullptr || ws_bytes < need))
+    return fail(TP_ENOSPACE, "workspace of %zu bytes < %zu needed", ws_bytes, need);
+  const EpiKind epi = c_dtype == TP_F32 ? EPI_F32 : EPI_BF16;
+  char* wsb = static_cast<char*>(ws);
+
+  if (case_id == 1) {                                   // X[B_X, D] . W[D, F]: local
+    if (strategy != TP_CASE1_LOCAL) return fail(TP_EINVAL, "case 1 has one strategy");
+    if (B % t) return fail(TP_EDIVIS, "t=%d does not divide B", t);
+    GemmArgs g = gemm_args(t, B / t, F, D, D, F, epi);
+    for (int i = 0; i < t; ++i) { g.a[i] = x[i]; g.b[i] = w[i]; g.c[i] = c[i]; }
+    return grouped_gemm(g, s);
+  }
+  if (case_id == 2) {                                   // X[B, D_X] . W[D, F]
+    if (D % t) return fail(TP_EDIVIS, "t=%d does not divide D", t);
+    if (strategy == TP_CASE2_ALLGATHER) {
+      const size_t slot = align256(size_t(B) * D * 2);
+      RingArgs ag = ring_args(RING_AG, t, B, D, 1, TP_BF16, TP_BF16);
+      for (int i = 0; i < t; ++i) { ag.in[i] = x[i]; ag.out[i] = wsb + i * slot; }
+      if (tp_status st = ring_collective(ag, s)) return st;
+      GemmArgs g = gemm_args(t, B, F, D, D, F, epi);
+      for (int i = 0; i < t; ++i) { g.a[i] = reinterpret_cast<const uint16_t*>(wsb + i * slot); g.b[i] = w[i]; g.c[i] = c[i]; }
+      return grouped_gemm(g, s);
+    }
+    if (strategy == TP_CASE2_ALLREDUCE) {
+      if (B % t) return fail(TP_EDIVIS, "t=%d does not divide B (AllReduce chunks)", t);
+      const size_t slot = align256(size_t(B) * F * 4);
+      const int64_t d = D / t;
+      GemmArgs g = gemm_args(t, B, F, d, d, F, EPI_F32);
+      for (int i = 0; i < t; ++i) { g.a[i] = x[i]; g.b[i] = w[i] + i * d * F; g.c[i] = wsb + i * slot; }
+      if (tp_status st = grouped_gemm(g, s)) return st;
+      RingArgs ar = ring_args(RING_AR, t, B, F, 0, TP_F32, c_dtype);
+      for (int i = 0; i < t; ++i) { ar.in[i] = wsb + i * slot; ar.out[i] = c[i]; }
+      return ring_collective(ar, s);
+    }
+    return fail(TP_EINVAL, "bad case-2 strategy %d", strategy);
+  }
+  if (case_id == 3) {                                   // X[B, D_X] . W[D_X, F] -> C{U_X}
+    if (D % t) return fail(TP_EDIVIS, "t=%d does not divide D", t);
+    if (strategy < TP_CASE3_ALLREDUCE || strategy > TP_CASE3_RS_F) return fail(TP_EINVAL, "bad case-3 strategy %d", strategy);
+    const size_t slot = align256(size_t(B) * F * 4);
+    const int64_t d = D / t;
+    GemmArgs g = gemm_args(t, B, F, d, d, F, EPI_F32);
+    for (int i = 0; i < t; ++i) { g.a[i] = x[i]; g.b[i] = w[i]; g.c[i] = wsb + i * slot; }
+    if (strategy == TP_CASE3_RS_F ? (F % t != 0) : (B % t != 0)) return fail(TP_EDIVIS, "t=%d does not divide the scattered dim", t);
+    if (tp_status st = grouped_gemm(g, s)) return st;
+    RingArgs a = ring_args(strategy == TP_CASE3_ALLREDUCE ? RING_AR : RING_RS, t, B, F,
+                           strategy == TP_CASE3_RS_F ? 1 : 0, TP_F32, c_dtype);
+    for (int i = 0; i < t; ++i) { a.in[i] = wsb + i * slot; a.out[i] = c[i]; }
+    return ring_collective(a, s);
+  }
+  if (case_id == 4) {                                   // X[B_X, D] . W[D, F_X]: gather one operand
+    if (B % t || F % t) return fail(TP_EDIVIS, "t=%d does not divide B and F", t);
+    if (strategy == TP_CASE4_GATHER_X) {
+      const size_t slot = align256(size_t(B) * D * 2);
+      RingArgs ag = ring_args(RING_AG, t, B, D, 0, TP_BF16, TP_BF16);
+      for (int i = 0; i < t; ++i) { ag.in[i] = x[i]; ag.out[i] = wsb + i * slot; }
+      if (tp_status st = ring_collective(ag, s)) return st;
+      GemmArgs g = gemm_args(t, B, F / t, D, D, F / t, epi);
+      for (int i = 0; i < t; ++i) { g.a[i] = reinterpret_cast<const uint16_t*>(wsb + i * slot); g.b[i] = w[i]; g.c[i] = c[i]; }
+      return grouped_gemm(g, s);
+    }
+    if (strategy == TP_CASE4_GATHER_W) {
+      const size_t slot = align256(size_t(D) * F * 2);
+      RingArgs ag = ring_args(RING_AG, t, D, F, 1, TP_BF16, TP_BF16);
+      for (int i = 0; i < t; ++i) { ag.in[i] = w[i]; ag.out[i] = wsb + i * slot; }
+      if (tp_status st = ring_collective(ag, s)) return st;
+      GemmArgs g = gemm_args(t, B / t, F, D, D, F, epi);
+      for (int i = 0; i < t; ++i) { g.a[i] = x[i]; g.b[i] = reinterpret_cast<const uint16_t*>(wsb + i * slot); g.c[i] = c[i]; }
+      return grouped_gemm(g, s);
+    }
+    return fail(TP_EINVAL, "bad case-4 strategy %d", strategy);
+  }
+  return fail(TP_EINVAL, "case_id %d outside 1..4", case_id);
+}
+
+tp_status tp_layer_fwd(const uint16_t* x, const uint16_t* const* o, int64_t N, int64_t h, int n_h, int n_kv, int d_h,
+                       int64_t F, int t, const uint16_t* w_qkv, const uint16_t* w_o, const uint16_t* w_gu,
+                       const uint16_t* w_down, uint16_t* qkv_out, float* const* h1, uint16_t* h1_bf16, uint16_t* z_ws,
+                       float* const* partials, float* const* y, void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (!valid_t(t)) return fail(TP_EINVAL, "t=%d outside 1..%d", t, TP_MAX_SHARDS);
+  if (!x || !o || !w_qkv || !w_o || !w_gu || !w_down || !qkv_out || !h1 || !h1_bf16 || !z_ws || !partials || !y)
+    return fail(TP_EINVAL, "null pointer");
+  if (N <= 0 || h <= 0 || F <= 0 || n_h <= 0 || n_kv <= 0 || d_h <= 0) return fail(TP_EINVAL, "non-positive size");
+  if (n_h % t || n_h % n_kv || (t <= n_kv ? n_kv % t != 0 : t % n_kv != 0))
+    return fail(TP_EDIVIS, "head counts n_h=%d n_kv=%d do not split over t=%d", n_h, n_kv, t);
+  if (F % t || N % t) return fail(TP_EDIVIS, "t=%d does not divide F or the token count", t);
+  const int64_t kv = t <= n_kv ? n_kv / t : 1;
+  const int64_t qkv_w = (n_h / t + 2 * kv) * d_h;
+  const int64_t o_w = int64_t(n_h) * d_h / t;
+  for (int r = 0; r < t; ++r)
+    if (o[r] == nullptr || h1[r] == nullptr || partials[r] == nullptr || y[r] == nullptr)
+      return fail(TP_EINVAL, "null shard buffer %d", r);
+  // 1. fused QKV projection, column-parallel on head boundaries (feeds the attention core)
+  if (tp_status st = column_gemm(x, N, h, qkv_w, t, TP_ACT_NONE, w_qkv, qkv_out, s)) return st;
+  // 2. attention output projection, row-parallel: partials O_r W_o[r]
+  {
+    GemmArgs g = gemm_args(t, N, h, o_w, o_w, h, EPI_F32);
+    for (int r = 0; r < t; ++r) { g.a[r] = o[r]; g.b[r] = w_o + r * o_w * h; g.c[r] = partials[r]; }
+    if (tp_status st = grouped_gemm(g, s)) return st;
+  }
+  // 3. g: AllReduce, fused with the residual add h1 = X + attn and the bf16 copy for the MLP input
+  if (tp_status st = reduce_partials(partials, N, h, t, TP_OUT_AR, h1, x, TP_BF16, h1_bf16, s)) return st;
+  // 4. SwiGLU MLP on bf16(h1), partials, then AllReduce fused with y = h1 + mlp
+  const int64_t f = F / t;
+  if (tp_status st = column_gemm(h1_bf16, N, h, f, t, TP_ACT_SWIGLU, w_gu, z_ws, s)) return st;
+  if (tp_status st = row_gemm(z_ws, N, f, h, t, w_down, partials, s)) return st;
+  return reduce_partials(partials, N, h, t, TP_OUT_AR, y, h1[0], TP_F32, nullptr, s);
+}
+
+}  // extern "C"

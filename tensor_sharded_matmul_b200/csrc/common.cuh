@@ -1,0 +1,66 @@
+// Host-side plumbing shared by the libtp translation units: error reporting, per-device caches,
+// argument checks. Device code lives in ptx.cuh and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "tp.h"
+
+namespace tpx {
+
+// Codes recorded in the device status word (which bounded wait ran out).
+enum WaitSite : uint32_t {
+  WAIT_SELFTEST = 1,
+  WAIT_PRODUCER_EMPTY = 2,   // TMA producer waiting for a free shared-memory stage
+  WAIT_MMA_FULL = 3,         // MMA issuer waiting for a stage's TMA bytes
+  WAIT_MMA_ACC_EMPTY = 4,    // MMA issuer waiting for the epilogue to drain an accumulator
+  WAIT_EPI_ACC_FULL = 5,     // epilogue waiting for an accumulator
+  WAIT_TEARDOWN = 6          // draining in-flight copies / MMAs before exit
+};
+
+// Records a failure message for the calling host thread and returns `s`.
+tp_status fail(tp_status s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+// Returns TP_ECUDA (with message) if the last launch failed, TP_OK otherwise.
+tp_status check_launch(const char* what);
+// Per-device address of the status word (nullptr when the runtime call fails).
+uint32_t* status_word();
+// Current budget of bounded device waits, in SM cycles.
+unsigned long long wait_budget();
+// Cached SM count of the current device (0 on failure).
+int sm_count();
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool valid_t(int t) { return t >= 1 && t <= TP_MAX_SHARDS; }
+
+// ---- internal entry points shared between translation units -------------------------------------
+enum RingOp { RING_RS = 0, RING_AG = 1, RING_AR = 2 };
+
+struct RingArgs {
+  RingOp op;
+  const void* in[TP_MAX_SHARDS];
+  void* out[TP_MAX_SHARDS];
+  tp_dtype in_dtype, out_dtype;
+  int64_t rows, cols;        // the full logical [rows, cols] matrix
+  int axis;                  // chunk axis (RS, AG)
+  int t;
+  const void* resid;         // AR only: optional residual added after the ring sum
+  tp_dtype resid_dtype;
+  uint16_t* copy_bf16;       // AR only: optional bf16 copy of the result (one buffer)
+};
+tp_status ring_collective(const RingArgs& a, cudaStream_t s);
+
+enum EpiKind { EPI_F32 = 0, EPI_BF16 = 1, EPI_GELU = 2, EPI_GELU_TANH = 3, EPI_SWIGLU = 4 };
+
+struct GemmArgs {
+  int groups;
+  const uint16_t* a[TP_MAX_SHARDS];  // [M, K] row-major, row stride lda elements
+  const uint16_t* b[TP_MAX_SHARDS];  // [K, Nb] row-major, row stride ldb (SwiGLU: [gate | up], up at +N)
+  void* c[TP_MAX_SHARDS];            // [M, N] row-major, row stride N
+  int64_t M, N, K, lda, ldb;
+  EpiKind epi;
+};
+tp_status grouped_gemm(const GemmArgs& g, cudaStream_t s);
+
+}  // namespace tpx

@@ -1,0 +1,110 @@
+"""The C ABI library loads, exports every entry point include/tp.h declares, and rejects bad
+arguments on the host before launching anything (CPU only: no call here reaches the GPU)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import tensor_sharded_matmul_b200 as tp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "tp.h")
+
+
+def declared_functions():
+    src = open(HEADER, encoding="utf-8").read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(tp_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for must in ("tp_shard_qkv", "tp_shard_gate_up", "tp_mlp_fwd", "tp_sharded_matmul", "tp_reduce_scatter",
+                 "tp_all_gather", "tp_all_reduce"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(tp.LIB_PATH)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+    out = subprocess.run(["nm", "-D", "--defined-only", tp.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (tp_\w+)", out))
+    assert set(declared_functions()) <= exported
+
+
+def test_binding_has_the_same_names():
+    assert set(declared_functions()) == set(tp.EXPORTED)
+    for n in declared_functions():
+        assert callable(getattr(tp, n))
+
+
+def test_status_strings():
+    assert tp.tp_status_str(tp.TP_OK) == "ok"
+    assert "divide" in tp.tp_status_str(tp.TP_EDIVIS)
+    assert tp.tp_status_str(99) == "unknown status"
+
+
+def _expect(status, fn, *args):
+    with pytest.raises(tp.TPError) as e:
+        fn(*args)
+    assert e.value.status == status, str(e.value)
+
+
+FAKE = 1 << 20   # a 16-byte aligned non-null address; never dereferenced (calls fail validation first)
+
+
+def test_collectives_validate_before_launch():
+    _expect(tp.TP_EINVAL, tp.tp_reduce_scatter, [FAKE] * 17, [FAKE] * 17, 16, 16, 0, tp.TP_F32, 17, 0)
+    _expect(tp.TP_EINVAL, tp.tp_reduce_scatter, [FAKE], [FAKE], 16, 16, 0, tp.TP_F32, 0, 0)
+    _expect(tp.TP_EDIVIS, tp.tp_reduce_scatter, [FAKE] * 3, [FAKE] * 3, 16, 16, 0, tp.TP_F32, 3, 0)
+    _expect(tp.TP_EDIVIS, tp.tp_all_gather, [FAKE] * 3, [FAKE] * 3, 16, 16, 1, tp.TP_BF16, 3, 0)
+    _expect(tp.TP_EINVAL, tp.tp_all_reduce, [FAKE, 0], [FAKE, FAKE], 16, 16, tp.TP_F32, 2, 0)
+    _expect(tp.TP_EINVAL, tp.tp_reduce_scatter, [FAKE] * 2, [FAKE] * 2, 16, 16, 2, tp.TP_F32, 2, 0)
+    _expect(tp.TP_EINVAL, tp.tp_reduce_scatter, [FAKE] * 2, [FAKE] * 2, 0, 16, 0, tp.TP_F32, 2, 0)
+
+
+def test_layouts_validate_before_launch():
+    _expect(tp.TP_EDIVIS, tp.tp_shard_cols, FAKE, 30, 8, 30, 4, FAKE, 0)
+    _expect(tp.TP_EDIVIS, tp.tp_shard_rows, FAKE, 8, 30, 8, 4, FAKE, 0)
+    _expect(tp.TP_EINVAL, tp.tp_shard_cols, FAKE, 8, 8, 16, 2, FAKE, 0)            # ld < N
+    # t must divide n_h; KV heads split (t | n_kv) or replicated (n_kv | t)
+    _expect(tp.TP_EDIVIS, tp.tp_shard_qkv, FAKE, 64, FAKE, 16, FAKE, 16, 64, 8, 2, 8, 3, FAKE, 0)
+    _expect(tp.TP_EDIVIS, tp.tp_shard_qkv, FAKE, 48, FAKE, 16, FAKE, 16, 64, 6, 2, 8, 4, FAKE, 0)  # 2 | 4 ok, 4 | 6 no
+    _expect(tp.TP_EDIVIS, tp.tp_shard_qkv, FAKE, 64, FAKE, 32, FAKE, 32, 64, 8, 4, 8, 16, FAKE, 0)  # t > n_h
+
+
+def test_gemm_and_mlp_validate_before_launch():
+    _expect(tp.TP_EALIGN, tp.tp_grouped_gemm, 1, [FAKE], [FAKE], [FAKE], 64, 64, 60, tp.TP_ACT_NONE, tp.TP_F32, 0)
+    _expect(tp.TP_EALIGN, tp.tp_grouped_gemm, 1, [FAKE + 8], [FAKE], [FAKE], 64, 64, 64, tp.TP_ACT_NONE, tp.TP_F32, 0)
+    _expect(tp.TP_EINVAL, tp.tp_grouped_gemm, 1, [FAKE], [FAKE], [FAKE], 64, 64, 64, tp.TP_ACT_GELU, tp.TP_F32, 0)
+    _expect(tp.TP_EINVAL, tp.tp_grouped_gemm, 0, [], [], [], 64, 64, 64, tp.TP_ACT_NONE, tp.TP_F32, 0)
+    _expect(tp.TP_EDIVIS, tp.tp_mlp_fwd, FAKE, 64, 256, 1000, 3, tp.TP_ACT_GELU, FAKE, FAKE, FAKE, [FAKE] * 3,
+            tp.TP_OUT_PARTIALS, None, 0)
+    _expect(tp.TP_EDIVIS, tp.tp_mlp_fwd, FAKE, 66, 256, 1024, 4, tp.TP_ACT_GELU, FAKE, FAKE, FAKE, [FAKE] * 4,
+            tp.TP_OUT_RS, [FAKE] * 4, 0)
+    _expect(tp.TP_EINVAL, tp.tp_mlp_fwd, FAKE, 64, 256, 1024, 4, 9, FAKE, FAKE, FAKE, [FAKE] * 4,
+            tp.TP_OUT_PARTIALS, None, 0)
+
+
+def test_sharded_matmul_workspace_sizes_and_validation():
+    B, D, F, t = 8192, 8192, 28672, 4
+    assert tp.tp_sharded_matmul_ws_bytes(1, 0, B, D, F, t) == 0
+    assert tp.tp_sharded_matmul_ws_bytes(2, tp.TP_CASE2_ALLGATHER, B, D, F, t) == t * B * D * 2
+    assert tp.tp_sharded_matmul_ws_bytes(2, tp.TP_CASE2_ALLREDUCE, B, D, F, t) == t * B * F * 4
+    assert tp.tp_sharded_matmul_ws_bytes(3, tp.TP_CASE3_RS_F, B, D, F, t) == t * B * F * 4
+    assert tp.tp_sharded_matmul_ws_bytes(4, tp.TP_CASE4_GATHER_W, B, D, F, t) == t * D * F * 2
+    _expect(tp.TP_ENOSPACE, tp.tp_sharded_matmul, 3, 0, [FAKE] * 4, [FAKE] * 4, 64, 64, 64, 4, [FAKE] * 4, tp.TP_F32,
+            FAKE, 10, 0)
+    _expect(tp.TP_EINVAL, tp.tp_sharded_matmul, 5, 0, [FAKE] * 4, [FAKE] * 4, 64, 64, 64, 4, [FAKE] * 4, tp.TP_F32,
+            FAKE, 1 << 30, 0)
+    _expect(tp.TP_EDIVIS, tp.tp_sharded_matmul, 3, 0, [FAKE] * 3, [FAKE] * 3, 64, 64, 64, 3, [FAKE] * 3, tp.TP_F32,
+            FAKE, 1 << 30, 0)
+
+
+def test_layer_validates_head_split():
+    args = [FAKE, [FAKE] * 3, 96, 256, 8, 2, 32, 768, 3, FAKE, FAKE, FAKE, FAKE, FAKE, [FAKE] * 3, FAKE, FAKE,
+            [FAKE] * 3, [FAKE] * 3, 0]
+    _expect(tp.TP_EDIVIS, tp.tp_layer_fwd, *args)

@@ -1,0 +1,256 @@
+"""GPU parity of the tensor-parallel MLP, the sharded-matmul cases and the tensor-parallel layer
+against the oracle, through the C ABI: the tiny GeLU MLP in full, the Llama-3-8B SwiGLU MLP, the
+four cases at B=D=8192, F=28672 and the Llama-3-70B-shaped layer at full size on sampled token rows
+(the oracle computes those rows one by one), plus GPU-side properties that hold at any size
+(AllReduce replicas identical, RS+AG == AR bit for bit, bf16 outputs = one rounding of fp32 outputs)."""
+import numpy as np
+import pytest
+import torch
+
+import synthetic as S
+import tensor_sharded_matmul_b200 as tp
+from gpu_util import GEMM_TOL, assert_close, cuda, f64, host_bits, same_bits
+from oracle import cases as OCASE
+from oracle import layer as OLAYER
+from oracle import layouts as OL
+from oracle import mlp as OM
+from oracle.bf16 import f32_to_bf16_bits
+
+pytestmark = pytest.mark.gpu
+
+
+def _status_ok():
+    st, site = tp.tp_device_status(1)
+    assert st == tp.TP_OK, f"device wait site {site}"
+
+
+def _mlp_device(X, w_in, w_down, N, h, F, t, act, mode):
+    f = F // t
+    z = torch.empty((t, N, f), dtype=torch.bfloat16, device="cuda")
+    partials = [torch.empty((N, h), device="cuda") for _ in range(t)]
+    if mode == tp.TP_OUT_RS:
+        out = [torch.empty((N // t, h), device="cuda") for _ in range(t)]
+    elif mode == tp.TP_OUT_PARTIALS:
+        out = None
+    else:
+        out = [torch.empty((N, h), device="cuda") for _ in range(t)]
+    tp.tp_mlp_fwd(X, N, h, F, t, act, w_in, w_down, z, partials, mode, out)
+    torch.cuda.synchronize()
+    _status_ok()
+    return z, partials, out
+
+
+# ---------------------------------------------------------------------------------- tiny GeLU MLP
+def test_tiny_gelu_mlp_all_modes():
+    N, h, F, t = 64, 256, 1024, 4
+    X, A, B = S.tiny_mlp(seed=0)
+    dX, dA, dB = cuda(X), cuda(A), cuda(B)
+    w_in = torch.empty((t, h, F // t), dtype=torch.bfloat16, device="cuda")
+    w_down = torch.empty((t, F // t, h), dtype=torch.bfloat16, device="cuda")
+    tp.tp_shard_cols(dA, F, h, F, t, w_in)
+    tp.tp_shard_rows(dB, h, F, h, t, w_down)
+    torch.cuda.synchronize()
+    Xf, Af, Bf = f64(X), f64(A), f64(B)
+    U = OM.mlp_partials(Xf, list(OL.shard_cols(Af, t)), list(OL.shard_rows(Bf, t)), "gelu")
+    Y = OM.mlp_unsharded(Xf, Af, Bf, "gelu")
+    results = {}
+    for mode in (tp.TP_OUT_PARTIALS, tp.TP_OUT_RS, tp.TP_OUT_AR, tp.TP_OUT_RS_AG):
+        z, partials, out = _mlp_device(dX, w_in, w_down, N, h, F, t, tp.TP_ACT_GELU, mode)
+        for r in range(t):
+            assert_close(f64(partials[r]), U[r], GEMM_TOL, f"partial {r}")
+        if mode == tp.TP_OUT_RS:
+            for r in range(t):
+                assert_close(f64(out[r]), Y[r * N // t:(r + 1) * N // t], GEMM_TOL, f"RS block {r}")
+        elif mode != tp.TP_OUT_PARTIALS:
+            for r in range(t):
+                assert_close(f64(out[r]), Y, GEMM_TOL, f"replica {r}")
+        results[mode] = (partials, out)
+    # GPU-side: AR replicas identical; RS+AG == AR; RS blocks == AR rows (same ring order, same partials)
+    ar = [host_bits(o) for o in results[tp.TP_OUT_AR][1]]
+    rsag = [host_bits(o) for o in results[tp.TP_OUT_RS_AG][1]]
+    rs = [host_bits(o) for o in results[tp.TP_OUT_RS][1]]
+    for r in range(t):
+        assert same_bits(ar[r], ar[0]) and same_bits(rsag[r], ar[0])
+        assert same_bits(rs[r], ar[0][r * N // t:(r + 1) * N // t])
+
+
+# ---------------------------------------------------------------------------------- Llama-3-8B SwiGLU MLP
+@pytest.fixture(scope="module")
+def llama8b():
+    N, h, F, t = 4096, 4096, 14336, 8
+    X, Wgu, Wd = S.llama8b_mlp(seed=0)
+    dX, dWgu, dWd = cuda(X), cuda(Wgu), cuda(Wd)
+    w_in = torch.empty((t, h, 2 * F // t), dtype=torch.bfloat16, device="cuda")
+    w_down = torch.empty((t, F // t, h), dtype=torch.bfloat16, device="cuda")
+    tp.tp_shard_gate_up(dWgu, 2 * F, dWgu.data_ptr() + 2 * F, 2 * F, h, F, t, w_in)
+    tp.tp_shard_rows(dWd, h, F, h, t, w_down)
+    torch.cuda.synchronize()
+    del dWgu, dWd
+    return dict(N=N, h=h, F=F, t=t, X=X, Wgu=Wgu, Wd=Wd, dX=dX, w_in=w_in, w_down=w_down)
+
+
+def test_llama8b_swiglu_mlp_sampled_rows(llama8b):
+    m = llama8b
+    N, h, F, t = m["N"], m["h"], m["F"], m["t"]
+    z, partials, out = _mlp_device(m["dX"], m["w_in"], m["w_down"], N, h, F, t, tp.TP_ACT_SWIGLU, tp.TP_OUT_RS_AG)
+    rows = np.sort(np.random.default_rng(0).choice(N, 48, replace=False))
+    Xr = f64(m["X"])[rows]
+    Wg = m["Wgu"][:, :F].float().numpy()
+    Wu = m["Wgu"][:, F:].float().numpy()
+    Wd = m["Wd"].float().numpy()
+    shards_in = list(OL.shard_gate_up(Wg, Wu, t))
+    shards_down = list(OL.shard_rows(Wd, t))
+    U = OM.mlp_partials(Xr, shards_in, shards_down, "swiglu")
+    Y = sum(U)
+    for r in (0, 3, 7):
+        assert_close(f64(partials[r])[rows], U[r], GEMM_TOL, f"partial {r}")
+    for s in range(t):
+        assert_close(f64(out[s])[rows], Y, GEMM_TOL, f"replica {s}")
+    # the activation workspace itself (Z_r = SiLU(X G_r) * X U_r) on the sampled rows
+    Z0 = OM.column_linear(Xr, shards_in[:1], "swiglu")[0]
+    assert_close(f64(z[0])[rows], Z0, GEMM_TOL, "Z_0")
+    # block identity on the device: the sum of the GPU partials equals the reduced output
+    total = sum(f64(p)[rows] for p in partials)
+    assert_close(f64(out[0])[rows], total, 1e-5, "sum of partials")
+
+
+def test_llama8b_modes_agree_bitwise(llama8b):
+    m = llama8b
+    N, h, F, t = m["N"], m["h"], m["F"], m["t"]
+    _, p1, ar = _mlp_device(m["dX"], m["w_in"], m["w_down"], N, h, F, t, tp.TP_ACT_SWIGLU, tp.TP_OUT_AR)
+    _, p2, rsag = _mlp_device(m["dX"], m["w_in"], m["w_down"], N, h, F, t, tp.TP_ACT_SWIGLU, tp.TP_OUT_RS_AG)
+    _, p3, rs = _mlp_device(m["dX"], m["w_in"], m["w_down"], N, h, F, t, tp.TP_ACT_SWIGLU, tp.TP_OUT_RS)
+    a0 = host_bits(ar[0])
+    for s in range(t):
+        assert same_bits(host_bits(ar[s]), a0)
+        assert same_bits(host_bits(rsag[s]), a0)
+        assert same_bits(host_bits(rs[s]), a0[s * N // t:(s + 1) * N // t])
+
+
+# ---------------------------------------------------------------------------------- sharded-matmul cases
+def _case_shards(X, W, case_id, t):
+    if case_id == 1:
+        return list(X.chunk(t, 0)), [W] * t
+    if case_id == 2:
+        return list(X.chunk(t, 1)), [W] * t
+    if case_id == 3:
+        return list(X.chunk(t, 1)), list(W.chunk(t, 0))
+    return list(X.chunk(t, 0)), list(W.chunk(t, 1))
+
+
+def _out_shape(case_id, strategy, B, F, t):
+    layout = OCASE.output_layout(case_id, OCASE.STRATEGIES[case_id][strategy])
+    return {"rows": (B // t, F), "cols": (B, F // t), "replicated": (B, F)}[layout], layout
+
+
+def _run_case(case_id, strategy, xs, ws, B, D, F, t, c_dtype):
+    shape, layout = _out_shape(case_id, strategy, B, F, t)
+    cdt = torch.float32 if c_dtype == tp.TP_F32 else torch.bfloat16
+    c = [torch.empty(shape, dtype=cdt, device="cuda") for _ in range(t)]
+    nbytes = tp.tp_sharded_matmul_ws_bytes(case_id, strategy, B, D, F, t)
+    ws_buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device="cuda")
+    tp.tp_sharded_matmul(case_id, strategy, xs, ws, B, D, F, t, c, c_dtype, ws_buf, nbytes)
+    torch.cuda.synchronize()
+    _status_ok()
+    return c, layout
+
+
+@pytest.mark.parametrize("case_id,strategy", [(1, 0), (2, 0), (2, 1), (3, 0), (3, 1), (3, 2), (4, 0), (4, 1)])
+def test_cases_small_against_oracle(case_id, strategy):
+    B, D, F, t = 512, 384, 768, 4
+    X, W = S.case_operands(seed=case_id, B=B, D=D, F=F)
+    xs, ws = _case_shards(X, W, case_id, t)
+    dxs = [cuda(x) for x in xs]
+    dws = [cuda(w) for w in ws]
+    ref = OCASE.run(case_id, OCASE.STRATEGIES[case_id][strategy], [f64(x) for x in xs], [f64(w) for w in ws])
+    c32, layout = _run_case(case_id, strategy, dxs, dws, B, D, F, t, tp.TP_F32)
+    c16, _ = _run_case(case_id, strategy, dxs, dws, B, D, F, t, tp.TP_BF16)
+    for i in range(t):
+        assert_close(f64(c32[i]), ref[i], GEMM_TOL, f"shard {i}")
+        assert_close(f64(c16[i]), ref[i], GEMM_TOL, f"shard {i} bf16")
+    logical = OCASE.to_logical([f64(c) for c in c32], layout)
+    assert_close(logical, f64(X) @ f64(W), GEMM_TOL, "logical C")
+    if layout == "replicated":
+        for i in range(t):
+            assert same_bits(host_bits(c32[i]), host_bits(c32[0]))
+    if case_id in (2, 3) and not (case_id == 2 and strategy == 0):
+        # reduced outputs: the bf16 result is the fp32 ring sum rounded once
+        for i in range(t):
+            assert np.array_equal(host_bits(c16[i]), f32_to_bf16_bits(host_bits(c32[i])))
+
+
+@pytest.fixture(scope="module")
+def case_operands_full():
+    X, W = S.case_operands(seed=0)
+    return X, W
+
+
+@pytest.mark.parametrize("case_id,strategy", [(1, 0), (2, 0), (2, 1), (3, 0), (3, 1), (3, 2), (4, 0), (4, 1)])
+def test_cases_full_size_sampled(case_operands_full, case_id, strategy):
+    B, D, F, t = 8192, 8192, 28672, 4
+    X, W = case_operands_full
+    xs, ws = _case_shards(X, W, case_id, t)
+    dxs = [cuda(x) for x in xs]
+    dws = [cuda(w) for w in ws] if case_id != 1 and case_id != 2 else [cuda(W)] * t
+    c, layout = _run_case(case_id, strategy, dxs, dws, B, D, F, t, tp.TP_F32)
+    g = np.random.default_rng(case_id * 10 + strategy)
+    rows = np.sort(g.choice(B, 24, replace=False))
+    cols = np.sort(g.choice(F, 96, replace=False))
+    ref = OM.matmul(f64(X[torch.from_numpy(rows)]), f64(W[:, torch.from_numpy(cols)]))
+    # gather the sampled logical entries from the shards
+    got = np.empty_like(ref)
+    for a, r in enumerate(rows):
+        for b, col in enumerate(cols):
+            if layout == "rows":
+                shard, rr, cc = r // (B // t), r % (B // t), col
+            elif layout == "cols":
+                shard, rr, cc = col // (F // t), r, col % (F // t)
+            else:
+                shard, rr, cc = (a + b) % t, r, col
+            got[a, b] = float(c[shard][rr, cc])
+    assert_close(got, ref, GEMM_TOL, f"case {case_id} strategy {strategy}")
+
+
+# ---------------------------------------------------------------------------------- 70B-shaped layer
+def test_llama70b_layer_sampled_rows():
+    N, h, n_h, n_kv, d_h, F, t = 2048, 8192, 64, 8, 128, 28672, 8
+    L = S.llama70b_layer(seed=0)
+    d = {k: cuda(v) for k, v in L.items()}
+    kv = n_kv // t
+    qkv_w = (n_h // t + 2 * kv) * d_h
+    w_qkv = torch.empty((t, h, qkv_w), dtype=torch.bfloat16, device="cuda")
+    w_o = torch.empty((t, n_h * d_h // t, h), dtype=torch.bfloat16, device="cuda")
+    w_gu = torch.empty((t, h, 2 * F // t), dtype=torch.bfloat16, device="cuda")
+    w_down = torch.empty((t, F // t, h), dtype=torch.bfloat16, device="cuda")
+    tp.tp_shard_qkv(d["Wq"], n_h * d_h, d["Wk"], n_kv * d_h, d["Wv"], n_kv * d_h, h, n_h, n_kv, d_h, t, w_qkv)
+    tp.tp_shard_rows(d["Wo"], h, n_h * d_h, h, t, w_o)
+    tp.tp_shard_gate_up(d["Wg"], F, d["Wu"], F, h, F, t, w_gu)
+    tp.tp_shard_rows(d["Wd"], h, F, h, t, w_down)
+    o_shards = [d["O"][:, r * n_h * d_h // t:(r + 1) * n_h * d_h // t].contiguous() for r in range(t)]
+    qkv_out = torch.empty((t, N, qkv_w), dtype=torch.bfloat16, device="cuda")
+    h1 = [torch.empty((N, h), device="cuda") for _ in range(t)]
+    h1_bf16 = torch.empty((N, h), dtype=torch.bfloat16, device="cuda")
+    z_ws = torch.empty((t, N, F // t), dtype=torch.bfloat16, device="cuda")
+    partials = [torch.empty((N, h), device="cuda") for _ in range(t)]
+    y = [torch.empty((N, h), device="cuda") for _ in range(t)]
+    tp.tp_layer_fwd(d["X"], o_shards, N, h, n_h, n_kv, d_h, F, t, w_qkv, w_o, w_gu, w_down, qkv_out, h1, h1_bf16,
+                    z_ws, partials, y)
+    torch.cuda.synchronize()
+    _status_ok()
+    rows = np.sort(np.random.default_rng(70).choice(N, 16, replace=False))
+    f32 = lambda x: x.float().numpy()  # noqa: E731  (exact widening of bf16)
+    sh_qkv = OL.shard_qkv(f32(L["Wq"]), f32(L["Wk"]), f32(L["Wv"]), n_h, n_kv, d_h, t)
+    sh_o = OL.shard_rows(f32(L["Wo"]), t)
+    sh_gu = OL.shard_gate_up(f32(L["Wg"]), f32(L["Wu"]), t)
+    sh_d = OL.shard_rows(f32(L["Wd"]), t)
+    O = f32(L["O"])
+    O_sh = [O[:, r * n_h * d_h // t:(r + 1) * n_h * d_h // t] for r in range(t)]
+    ref = OLAYER.layer_forward(f32(L["X"]), O_sh, list(sh_qkv), list(sh_o), list(sh_gu), list(sh_d), rows=rows)
+    for r in (0, 5):
+        assert_close(f64(qkv_out[r])[rows], ref["qkv"][r], GEMM_TOL, f"qkv {r}")
+    assert_close(f64(h1[3])[rows], ref["h1"], GEMM_TOL, "h1")
+    for s in (0, 7):
+        assert_close(f64(y[s])[rows], ref["y"], GEMM_TOL, f"y replica {s}")
+        assert same_bits(host_bits(y[s]), host_bits(y[0]))
+    # the MLP contribution alone, y - h1, against the oracle's
+    assert_close(f64(y[0])[rows] - f64(h1[0])[rows], ref["mlp"], GEMM_TOL, "mlp part")
