@@ -15,7 +15,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libtp.so")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m tensor_sharded_matmul_b200.build` "
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python tensor_sharded_matmul_b200/build.py` "
                       "(or __graft_entry__.build()); there is no fallback implementation")
 
 _lib = C.CDLL(LIB_PATH)

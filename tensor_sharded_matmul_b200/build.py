@@ -1,6 +1,8 @@
 """Builds libtp.so in-tree from csrc/*.cu with nvcc for sm_100a (B200).
 
-    python -m tensor_sharded_matmul_b200.build [--force] [--jobs N]
+    python tensor_sharded_matmul_b200/build.py [--force] [--jobs N]
+
+(run it as a script: importing the package loads libtp.so, which this script is what builds)
 
 Objects go to <repo>/_build/, the shared library to tensor_sharded_matmul_b200/libtp.so. The CUDA
 runtime is linked statically, so the library needs only the NVIDIA driver at run time.
