@@ -212,6 +212,29 @@ tp_status tp_layer_fwd(const uint16_t* x, const uint16_t* const* o, int64_t N, i
                        const uint16_t* w_gu, const uint16_t* w_down, uint16_t* qkv_out, float* const* h1,
                        uint16_t* h1_bf16, uint16_t* z_ws, float* const* partials, float* const* y, void* stream);
 
+/* ------------------------------------------------------------------------------------------------
+ * tp_mlp_fwd without caller-provided scratch. The pages have no counterpart: this entry point exists
+ * for callers that cannot allocate device memory. Examples are code inside a host framework whose
+ * caching pool owns the GPU's memory, where an allocation behind the pool's back can fail or escape
+ * its accounting, and serving loops that forbid cudaMalloc/cudaFree after start-up because those
+ * calls can synchronise the device.
+ * Same computation, arguments and results as tp_mlp_fwd, minus z_ws and partials. The activations
+ * and the fp32 partials live in one array of TP_MLP_NOALLOC_SCRATCH_BYTES compiled into the library,
+ * which every GPU that loads the library holds until the process exits.
+ *   - Requests needing more than that (N*F*2 bytes, plus t*N*h*4 unless mode is TP_OUT_PARTIALS, each
+ *     rounded up to 256) return TP_ENOSPACE before any launch.
+ *   - In TP_OUT_PARTIALS mode the partials are written to out[] (t fp32 [N, h] buffers).
+ *   - All calls share the array and it keeps the last call's contents; every call overwrites all
+ *     the scratch it reads, so nothing needs clearing. Calls that overlap on the GPU race on it.
+ *   - The first call on a device resolves the array's address (it may load the module); make it
+ *     before any stream capture.
+ *   - No cudaMalloc, cudaFree or allocating library routine is called.
+ * ------------------------------------------------------------------------------------------------ */
+#define TP_MLP_NOALLOC_SCRATCH_BYTES (32u << 20)
+tp_status tp_mlp_fwd_noalloc(const uint16_t* x, int64_t N, int64_t h, int64_t F, int t, tp_act act,
+                             const uint16_t* w_in, const uint16_t* w_down, tp_reduce mode, float* const* out,
+                             void* stream);
+
 #ifdef __cplusplus
 }
 #endif

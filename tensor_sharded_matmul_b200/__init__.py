@@ -35,7 +35,7 @@ EXPORTED = (
     "tp_status_str", "tp_last_error", "tp_device_status", "tp_set_wait_budget", "tp_selftest_wait_timeout",
     "tp_num_sms", "tp_shard_cols", "tp_shard_rows", "tp_shard_gate_up", "tp_shard_qkv", "tp_reduce_scatter",
     "tp_all_gather", "tp_all_reduce", "tp_grouped_gemm", "tp_column_linear", "tp_row_linear", "tp_mlp_fwd",
-    "tp_sharded_matmul_ws_bytes", "tp_sharded_matmul", "tp_layer_fwd",
+    "tp_sharded_matmul_ws_bytes", "tp_sharded_matmul", "tp_layer_fwd", "tp_mlp_fwd_noalloc",
 )
 
 _vp, _i64, _i32, _u64, _sz = C.c_void_p, C.c_int64, C.c_int, C.c_uint64, C.c_size_t
@@ -59,6 +59,7 @@ _SIGS = {
     "tp_column_linear": (_i32, [_vp, _i64, _i64, _i64, _i32, _i32, _vp, _vp, _vp]),
     "tp_row_linear": (_i32, [_vp, _i64, _i64, _i64, _i32, _vp, _pp, _vp]),
     "tp_mlp_fwd": (_i32, [_vp, _i64, _i64, _i64, _i32, _i32, _vp, _vp, _vp, _pp, _i32, _pp, _vp]),
+    "tp_mlp_fwd_noalloc": (_i32, [_vp, _i64, _i64, _i64, _i32, _i32, _vp, _vp, _i32, _pp, _vp]),
     "tp_sharded_matmul_ws_bytes": (_sz, [_i32, _i32, _i64, _i64, _i64, _i32]),
     "tp_sharded_matmul": (_i32, [_i32, _i32, _pp, _pp, _i64, _i64, _i64, _i32, _pp, _i32, _vp, _sz, _vp]),
     "tp_layer_fwd": (_i32, [_vp, _pp, _i64, _i64, _i32, _i32, _i32, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _pp,
@@ -183,6 +184,16 @@ def tp_row_linear(x, N, k, n, t, w, partials, stream=None):
 def tp_mlp_fwd(x, N, h, F, t, act, w_in, w_down, z_ws, partials, mode, out, stream=None):
     _call("tp_mlp_fwd", _ptr(x), N, h, F, t, act, _ptr(w_in), _ptr(w_down), _ptr(z_ws), _ptrs(partials), mode,
           _ptrs(out), _stream(stream))
+
+
+def tp_mlp_fwd_noalloc(x, N, h, F, t, act, w_in, w_down, mode, out, stream=None):
+    """tp_mlp_fwd for callers that cannot allocate device memory: the scratch is a fixed array inside
+    the library (TP_MLP_NOALLOC_SCRATCH_BYTES); see include/tp.h for its limits and sharing rules."""
+    _call("tp_mlp_fwd_noalloc", _ptr(x), N, h, F, t, act, _ptr(w_in), _ptr(w_down), mode, _ptrs(out),
+          _stream(stream))
+
+
+TP_MLP_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 def tp_sharded_matmul_ws_bytes(case_id, strategy, B, D, F, t) -> int:
