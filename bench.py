@@ -2,15 +2,18 @@
 
 One step = one full pass of the hot path on the Llama-3-8B-shaped SwiGLU MLP, t=8 virtual shards:
   column-parallel GEMM + SwiGLU epilogue (Z_r = SiLU(X G_r) * X U_r)
-  -> row-parallel GEMM (fp32 partials U_r = Z_r W_down[r])
-  -> ring ReduceScatter along tokens -> in-place AllGather (the config's AllReduce as RS then AG).
+  -> row-parallel GEMM with its ring ReduceScatter along tokens and the AllGather fused into the
+     epilogue (tp_row_linear_reduce, TP_OUT_RS_AG): the partials U_r = Z_r W_down[r] are summed in
+     ring order inside the kernel and each reduced tile is written to every shard.
+The standalone ring ReduceScatter (the second half of the metric) is timed in its own loop on the
+same data volume: 8 fp32 partials [4096, 4096].
 X [4096, 4096] bf16 ~N(0,1); fused gate|up [4096, 2*14336] and W_down [14336, 4096] ~N(0, 0.02), drawn
 on the device from a seeded generator, sharded once by the library's layout kernels (not timed).
 
 Output: one JSON line (rank 0). value = whole-job TFLOP/s (algorithmic FLOPs 2*N*h*F*2 + 2*N*F*h per
 step per replica, summed over replicas / max-over-ranks time). Per-kernel CUDA-event times inside the
-timed region give the roofline of the dominant kernel (the column GEMM, tensor-bound) and of the
-ReduceScatter (HBM-bound, algorithmic bytes (t+1)*M). `e2e` repeats the step through tp_mlp_fwd with
+timed region give the roofline of the dominant kernel (the column GEMM, tensor-bound); the standalone
+ReduceScatter loop gives the HBM roofline (algorithmic bytes (t+1)*M). `e2e` repeats the step through tp_mlp_fwd with
 X copied in from pinned host memory and the result copied back, every step. `cpu_baseline` times the
 oracle on a bounded row sample of the same workload on this host.
 
@@ -42,7 +45,7 @@ M_PARTIAL = N_TOK * H * 4                       # one fp32 partial, 64 MiB
 RS_BYTES = (T + 1) * M_PARTIAL                  # read t*M, write M
 AG_BYTES = T * M_PARTIAL                        # in place: read M once, write the t-1 other copies
 WORKLOAD = ("llama3-8b SwiGLU TP-MLP forward, t=8 virtual shards, 4096 tokens x h=4096, F=14336; "
-            "column GEMM+SwiGLU -> row GEMM (fp32 partials) -> ring ReduceScatter(tokens) -> AllGather")
+            "column GEMM+SwiGLU -> row GEMM fused with ring ReduceScatter(tokens) + AllGather")
 CPU_SAMPLE_ROWS = 512
 REF_ROWS_PER_STEP = 64
 
@@ -129,6 +132,23 @@ def _dist_env():
 
 def _emit(obj):
     print(json.dumps(obj), flush=True)
+
+
+def max_over_ranks(values, dist=None, device=None):
+    """Element-wise maximum over all ranks of a list of per-rank timings (identity for one process).
+    Every rank must call it with the same number of values, at the same point."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def whole_job_rate(work_per_step: float, steps: int, n_ranks: int, max_ms: float) -> float:
+    """Throughput of the whole job: every rank processes `work_per_step` per step (weak scaling), the
+    job lasts as long as its slowest rank."""
+    return n_ranks * work_per_step * steps / (max_ms * 1e-3)
 
 
 # ------------------------------------------------------------------------------ CPU oracle timing
@@ -233,28 +253,18 @@ def run_gpu(args) -> int:
     tp.tp_shard_rows(Wd, H, F, H, T, w_down)
     del Wgu, Wd
     z = torch.empty((T, N_TOK, f), dtype=torch.bfloat16, device=dev)
-    partials = [torch.empty((N_TOK, H), device=dev) for _ in range(T)]
     out = [torch.empty((N_TOK, H), device=dev) for _ in range(T)]
-    chunk = N_TOK // T
-    rs_blocks = [out[r][r * chunk:(r + 1) * chunk] for r in range(T)]
-    p_ptrs = partials
 
     def step(ev=None):
-        # exactly tp_mlp_fwd(..., TP_OUT_RS_AG), split at its kernel boundaries so each launch is timed
+        # exactly tp_mlp_fwd(..., TP_OUT_RS_AG), split at its kernel boundary so each launch is timed
         if ev is not None:
             ev[0].record(stream)
         tp.tp_column_linear(X, N_TOK, H, F, T, tp.TP_ACT_SWIGLU, w_in, z)
         if ev is not None:
             ev[1].record(stream)
-        tp.tp_row_linear(z, N_TOK, F, H, T, w_down, p_ptrs)
+        tp.tp_row_linear_reduce(z, N_TOK, F, H, T, w_down, tp.TP_OUT_RS_AG, 0, out)
         if ev is not None:
             ev[2].record(stream)
-        tp.tp_reduce_scatter(p_ptrs, rs_blocks, N_TOK, H, 0, tp.TP_F32, T)
-        if ev is not None:
-            ev[3].record(stream)
-        tp.tp_all_gather(rs_blocks, out, N_TOK, H, 0, tp.TP_F32, T)
-        if ev is not None:
-            ev[4].record(stream)
 
     for _ in range(args.warmup):
         step()
@@ -274,7 +284,7 @@ def run_gpu(args) -> int:
     if rank == 0:
         clocks.start()
         time.sleep(0.3)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if dist:
         dist.barrier()
@@ -292,8 +302,25 @@ def run_gpu(args) -> int:
     if st != tp.TP_OK:
         print(f"device wait ran out at site {site}", file=sys.stderr)
         return 3
-    per = [[evs[i][k].elapsed_time(evs[i][k + 1]) for i in range(args.steps)] for k in range(4)]
-    avg = [sum(p) / len(p) for p in per]      # ms: column GEMM, row GEMM, RS, AG
+    per = [[evs[i][k].elapsed_time(evs[i][k + 1]) for i in range(args.steps)] for k in range(2)]
+    avg = [sum(p) / len(p) for p in per]      # ms: column GEMM, fused row GEMM + RS + AG
+
+    # ---- the standalone ring ReduceScatter on the same volume (8 fp32 partials [4096, 4096]) -----
+    partials = [torch.empty((N_TOK, H), device=dev).normal_() for _ in range(T)]
+    chunk = N_TOK // T
+    rs_out = [torch.empty((chunk, H), device=dev) for _ in range(T)]
+    for _ in range(3):
+        tp.tp_reduce_scatter(partials, rs_out, N_TOK, H, 0, tp.TP_F32, T)
+    rs_start, rs_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    rs_iters = max(args.steps, 20)
+    torch.cuda.synchronize()
+    rs_start.record(stream)
+    for _ in range(rs_iters):
+        tp.tp_reduce_scatter(partials, rs_out, N_TOK, H, 0, tp.TP_F32, T)
+    rs_stop.record(stream)
+    torch.cuda.synchronize()
+    rs_ms = rs_start.elapsed_time(rs_stop) / rs_iters
+    del partials, rs_out
 
     # ---- end to end through tp_mlp_fwd with host buffers --------------------------------------
     x_host = X.cpu().pin_memory()
@@ -301,7 +328,7 @@ def run_gpu(args) -> int:
     x_dev = torch.empty_like(X)
     for _ in range(max(1, min(args.warmup, 3))):
         x_dev.copy_(x_host, non_blocking=True)
-        tp.tp_mlp_fwd(x_dev, N_TOK, H, F, T, tp.TP_ACT_SWIGLU, w_in, w_down, z, p_ptrs, tp.TP_OUT_RS_AG, out)
+        tp.tp_mlp_fwd(x_dev, N_TOK, H, F, T, tp.TP_ACT_SWIGLU, w_in, w_down, z, None, tp.TP_OUT_RS_AG, out)
         y_host.copy_(out[0], non_blocking=True)
     e_start, e_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if dist:
@@ -310,40 +337,41 @@ def run_gpu(args) -> int:
     e_start.record(stream)
     for _ in range(args.steps):
         x_dev.copy_(x_host, non_blocking=True)
-        tp.tp_mlp_fwd(x_dev, N_TOK, H, F, T, tp.TP_ACT_SWIGLU, w_in, w_down, z, p_ptrs, tp.TP_OUT_RS_AG, out)
+        tp.tp_mlp_fwd(x_dev, N_TOK, H, F, T, tp.TP_ACT_SWIGLU, w_in, w_down, z, None, tp.TP_OUT_RS_AG, out)
         y_host.copy_(out[0], non_blocking=True)
     e_stop.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e_start.elapsed_time(e_stop)
 
     # ---- max over ranks ------------------------------------------------------------------------
-    if dist:
-        tt = torch.tensor([total_ms, e2e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms, e2e_ms = float(tt[0]), float(tt[1])
+    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dist, dev)
     n = ws
     per_step_ms = total_ms / args.steps
-    value = n * FLOPS_STEP * args.steps / (total_ms * 1e-3) / 1e12
-    e2e_value = n * FLOPS_STEP * args.steps / (e2e_ms * 1e-3) / 1e12
+    value = whole_job_rate(FLOPS_STEP, args.steps, n, total_ms) / 1e12
+    e2e_value = whole_job_rate(FLOPS_STEP, args.steps, n, e2e_ms) / 1e12
 
     if rank == 0:
         hbm, bf16_burst, bf16_sust, src = _peaks()
         long_region = total_ms > 1000.0
         gemm_peak = bf16_sust if long_region else bf16_burst
         col_tflops = FLOPS_COL / (avg[0] * 1e-3) / 1e12
-        rs_gbs = RS_BYTES / (avg[2] * 1e-3) / 1e9
+        rs_gbs = RS_BYTES / (rs_ms * 1e-3) / 1e9
         roofline = {"bound": "tensor", "kernel": "gemm_tcgen05_kernel<SwiGLU> (column-parallel gate|up GEMM)",
                     "achieved": col_tflops, "peak": gemm_peak, "unit": "TFLOP/s", "frac": col_tflops / gemm_peak,
                     "peak_source": f"{src} bf16 {'sustained' if long_region else 'burst'}",
                     "flops_per_launch": FLOPS_COL, "avg_launch_ms": avg[0],
                     "traffic": _traffic("gemm_swiglu_8b", "gemm.cu")}
-        roofline_rs = {"bound": "hbm", "kernel": "ring_reduce_kernel<f32,t=8> (ReduceScatter along tokens)",
+        roofline_rs = {"bound": "hbm", "kernel": "ring_reduce_kernel<f32,t=8> (standalone ReduceScatter along tokens)",
                        "achieved": rs_gbs, "peak": hbm, "unit": "GB/s", "frac": rs_gbs / hbm,
-                       "peak_source": f"{src} hbm copy", "bytes_per_launch": RS_BYTES, "avg_launch_ms": avg[2],
-                       "bus_bw_gbs": (T - 1) / T * M_PARTIAL / (avg[2] * 1e-3) / 1e9,
+                       "peak_source": f"{src} hbm copy", "bytes_per_launch": RS_BYTES, "avg_launch_ms": rs_ms,
+                       "bus_bw_gbs": (T - 1) / T * M_PARTIAL / (rs_ms * 1e-3) / 1e9,
                        "traffic": _traffic("ring_rs_f32_t8", "collectives.cu")}
         row_tflops = FLOPS_ROW / (avg[1] * 1e-3) / 1e12
-        ag_gbs = AG_BYTES / (avg[3] * 1e-3) / 1e9
+        fused_roof = {"bound": "tensor", "kernel": "gemm_ring_kernel<f32,AR> (row GEMM + ring RS + AG)",
+                      "achieved": row_tflops, "peak": gemm_peak, "unit": "TFLOP/s", "frac": row_tflops / gemm_peak,
+                      "flops_per_launch": FLOPS_ROW, "avg_launch_ms": avg[1],
+                      "bytes_written_per_launch": T * M_PARTIAL,
+                      "traffic": _traffic("gemm_ring_8b", "gemm.cu")}
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": n, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": per_step_ms, "higher_is_better": True, "scaling": "weak",
@@ -353,14 +381,14 @@ def run_gpu(args) -> int:
                        "l2": "no flush: each step touches ~1.5 GB (weights 336 MiB, partials and outputs 1 GiB) > 126 MB L2"},
             "frac_of_peak_bf16": value / n / gemm_peak,
             "reduce_scatter": {"value": rs_gbs, "unit": "GB/s", "frac_hbm": rs_gbs / hbm},
-            "kernels_ms": {"column_gemm_swiglu": avg[0], "row_gemm_f32": avg[1], "reduce_scatter": avg[2],
-                           "all_gather_in_place": avg[3]},
-            "kernels_rate": {"column_gemm_tflops": col_tflops, "row_gemm_tflops": row_tflops,
-                             "reduce_scatter_gbs": rs_gbs, "all_gather_gbs": ag_gbs},
-            "roofline": roofline, "roofline_reduce_scatter": roofline_rs,
+            "kernels_ms": {"column_gemm_swiglu": avg[0], "row_gemm_rs_ag_fused": avg[1],
+                           "standalone_reduce_scatter": rs_ms},
+            "kernels_rate": {"column_gemm_tflops": col_tflops, "row_gemm_fused_tflops": row_tflops,
+                             "reduce_scatter_gbs": rs_gbs},
+            "roofline": roofline, "roofline_fused_row_reduce": fused_roof, "roofline_reduce_scatter": roofline_rs,
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": X.numel() * 2,
                     "d2h_bytes_per_step": N_TOK * H * 4},
-            "gpu_launches": 4 * args.steps,
+            "gpu_launches": 2 * args.steps,
             "clocks": clk,
         }
         if not args.no_cpu_baseline:

@@ -161,6 +161,21 @@ tp_status tp_column_linear(const uint16_t* x, int64_t N, int64_t k, int64_t n, i
 tp_status tp_row_linear(const uint16_t* x, int64_t N, int64_t k, int64_t n, int t, const uint16_t* w,
                         float* const* partials, void* stream);
 
+/* Row-parallel linear fused with its collective: the one-GPU form of collective matmul ([CH06] §6.6;
+ * [TPSP] §把通信藏到计算后面). out = Reduce_r(x[r] . w[r]) with x stacked [t][N][k/t] and w stacked
+ * [t][k/t][n], without materialising the fp32 partials. The kernel computes each output tile's t
+ * shard products in ring order (c+1, ..., c for the tile's chunk c), accumulates them in binary32
+ * exactly as tp_reduce_scatter would, and writes the tile once:
+ *   TP_OUT_RS           out[r] receives chunk r: [N/t, n] (axis 0) or [N, n/t] (axis 1)
+ *   TP_OUT_AR, RS_AG    every out[r] receives the whole [N, n] sum (ReduceScatter with its AllGather
+ *                       folded into the same epilogue; bit-identical to tp_all_reduce)
+ * Results are bit-identical to tp_row_linear followed by tp_reduce_scatter / tp_all_reduce.
+ * The fused kernel needs (N/t) % 128 == 0 for axis 0, or (n/t) % 256 == 0 for axis 1. Otherwise
+ * `partials` (t fp32 [N, n] buffers, else NULL) is used for the unfused path, and without it the
+ * call returns TP_EUNSUPPORTED. Aligned; k/t and n multiples of 8. */
+tp_status tp_row_linear_reduce(const uint16_t* x, int64_t N, int64_t k, int64_t n, int t, const uint16_t* w,
+                               tp_reduce mode, int axis, float* const* out, float* const* partials, void* stream);
+
 /* ------------------------------------------------------------------------------------------------
  * The tensor-parallel MLP forward ([TPSP] §MLP：先列后行，只通信一次; [PFY] §Tensor Parallel;
  * [CH06] §6.9 Problem 5): Z_r = act(X W_in[r]) (column-parallel, local), U_r = Z_r W_down[r]
@@ -169,7 +184,9 @@ tp_status tp_row_linear(const uint16_t* x, int64_t N, int64_t k, int64_t n, int 
  *   w_in    bf16 stacked [t][h][F/t] (GELU/NONE) or [t][h][2F/t] (SWIGLU, from tp_shard_gate_up)
  *   w_down  bf16 stacked [t][F/t][h] (from tp_shard_rows)
  *   z_ws    bf16 workspace [t][N][F/t] (the activations Z_r)
- *   partials t fp32 [N, h] buffers (the {U}); required for every mode
+ *   partials t fp32 [N, h] buffers (the {U}): the result in TP_OUT_PARTIALS mode. The reducing modes
+ *           fuse the row GEMM with its collective (tp_row_linear_reduce) whenever (N/t) % 128 == 0,
+ *           and then never touch partials, which may be NULL. Otherwise they are scratch.
  *   out     t fp32 buffers: unused for PARTIALS; [N/t, h] for RS (t | N); [N, h] for AR and RS_AG
  * Aligned; h and F/t multiples of 8. */
 tp_status tp_mlp_fwd(const uint16_t* x, int64_t N, int64_t h, int64_t F, int t, tp_act act,
@@ -205,7 +222,9 @@ tp_status tp_sharded_matmul(int case_id, int strategy, const uint16_t* const* x,
  *   w_gu   bf16 stacked [t][h][2F/t];  w_down bf16 stacked [t][F/t][h]
  *   qkv_out bf16 stacked [t][N][(n_h/t + 2kv)*d_h]
  *   h1     t fp32 [N, h] (replicas of the residual stream after attention); h1_bf16 bf16 [N, h]
- *   z_ws   bf16 [t][N][F/t]; partials t fp32 [N, h]; y t fp32 [N, h]
+ *   z_ws   bf16 [t][N][F/t]; y t fp32 [N, h]
+ *   partials t fp32 [N, h] scratch, needed only when (N/t) % 128 != 0; otherwise both row GEMMs are
+ *          fused with their AllReduce (and residual) and partials may be NULL
  * ------------------------------------------------------------------------------------------------ */
 tp_status tp_layer_fwd(const uint16_t* x, const uint16_t* const* o, int64_t N, int64_t h, int n_h, int n_kv,
                        int d_h, int64_t F, int t, const uint16_t* w_qkv, const uint16_t* w_o,

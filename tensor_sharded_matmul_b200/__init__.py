@@ -34,7 +34,7 @@ TP_MAX_SHARDS = 16
 EXPORTED = (
     "tp_status_str", "tp_last_error", "tp_device_status", "tp_set_wait_budget", "tp_selftest_wait_timeout",
     "tp_num_sms", "tp_shard_cols", "tp_shard_rows", "tp_shard_gate_up", "tp_shard_qkv", "tp_reduce_scatter",
-    "tp_all_gather", "tp_all_reduce", "tp_grouped_gemm", "tp_column_linear", "tp_row_linear", "tp_mlp_fwd",
+    "tp_all_gather", "tp_all_reduce", "tp_grouped_gemm", "tp_column_linear", "tp_row_linear", "tp_row_linear_reduce", "tp_mlp_fwd",
     "tp_sharded_matmul_ws_bytes", "tp_sharded_matmul", "tp_layer_fwd", "tp_mlp_fwd_noalloc",
 )
 
@@ -58,6 +58,7 @@ _SIGS = {
     "tp_grouped_gemm": (_i32, [_i32, _pp, _pp, _pp, _i64, _i64, _i64, _i32, _i32, _vp]),
     "tp_column_linear": (_i32, [_vp, _i64, _i64, _i64, _i32, _i32, _vp, _vp, _vp]),
     "tp_row_linear": (_i32, [_vp, _i64, _i64, _i64, _i32, _vp, _pp, _vp]),
+    "tp_row_linear_reduce": (_i32, [_vp, _i64, _i64, _i64, _i32, _vp, _i32, _i32, _pp, _pp, _vp]),
     "tp_mlp_fwd": (_i32, [_vp, _i64, _i64, _i64, _i32, _i32, _vp, _vp, _vp, _pp, _i32, _pp, _vp]),
     "tp_mlp_fwd_noalloc": (_i32, [_vp, _i64, _i64, _i64, _i32, _i32, _vp, _vp, _i32, _pp, _vp]),
     "tp_sharded_matmul_ws_bytes": (_sz, [_i32, _i32, _i64, _i64, _i64, _i32]),
@@ -179,6 +180,11 @@ def tp_column_linear(x, N, k, n, t, act, w, y, stream=None):
 
 def tp_row_linear(x, N, k, n, t, w, partials, stream=None):
     _call("tp_row_linear", _ptr(x), N, k, n, t, _ptr(w), _ptrs(partials), _stream(stream))
+
+
+def tp_row_linear_reduce(x, N, k, n, t, w, mode, axis, out, partials=None, stream=None):
+    _call("tp_row_linear_reduce", _ptr(x), N, k, n, t, _ptr(w), mode, axis, _ptrs(out), _ptrs(partials),
+          _stream(stream))
 
 
 def tp_mlp_fwd(x, N, h, F, t, act, w_in, w_down, z_ws, partials, mode, out, stream=None):

@@ -93,6 +93,27 @@ tp_status reduce_partials(float* const* partials, int64_t N, int64_t h, int t, t
   return fail(TP_EINVAL, "bad reduce mode %d", static_cast<int>(mode));
 }
 
+// Row-parallel GEMM fused with its collective (see gemm.cu): RS leaves chunk r on out[r]; AR and
+// RS_AG (ReduceScatter with its AllGather folded into the same epilogue) write every replica.
+tp_status fused_row_reduce(const uint16_t* x, int64_t N, int64_t k_shard, int64_t n, int t, const uint16_t* w,
+                           tp_reduce mode, int axis, float* const* out, const void* resid, tp_dtype resid_dtype,
+                           uint16_t* copy_bf16, cudaStream_t s) {
+  RingGemmArgs g;
+  std::memset(&g, 0, sizeof(g));
+  g.t = t; g.M = N; g.N = n; g.K = k_shard; g.lda = k_shard; g.ldb = n;
+  g.op = mode == TP_OUT_RS ? RING_RS : RING_AR;
+  g.axis = axis;
+  g.out_dtype = TP_F32;
+  g.resid = resid; g.resid_dtype = resid_dtype; g.copy_bf16 = copy_bf16;
+  for (int r = 0; r < t; ++r) {
+    if (out[r] == nullptr) return fail(TP_EINVAL, "null output buffer %d", r);
+    g.a[r] = x + r * N * k_shard;
+    g.b[r] = w + r * k_shard * n;
+    g.out[r] = out[r];
+  }
+  return ring_gemm(g, s);
+}
+
 }  // namespace
 }  // namespace tpx
 
@@ -130,13 +151,35 @@ tp_status tp_row_linear(const uint16_t* x, int64_t N, int64_t k, int64_t n, int 
   return row_gemm(x, N, k / t, n, t, w, partials, static_cast<cudaStream_t>(stream));
 }
 
+tp_status tp_row_linear_reduce(const uint16_t* x, int64_t N, int64_t k, int64_t n, int t, const uint16_t* w,
+                               tp_reduce mode, int axis, float* const* out, float* const* partials, void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (!valid_t(t)) return fail(TP_EINVAL, "t=%d outside 1..%d", t, TP_MAX_SHARDS);
+  if (x == nullptr || w == nullptr || out == nullptr) return fail(TP_EINVAL, "null pointer");
+  if (N <= 0 || k <= 0 || n <= 0) return fail(TP_EINVAL, "non-positive size");
+  if (mode != TP_OUT_RS && mode != TP_OUT_AR && mode != TP_OUT_RS_AG) return fail(TP_EINVAL, "mode must reduce");
+  if (axis != 0 && axis != 1) return fail(TP_EINVAL, "axis must be 0 or 1");
+  if (mode != TP_OUT_RS) axis = 0;
+  if (k % t) return fail(TP_EDIVIS, "t=%d does not divide k=%lld", t, (long long)k);
+  if (axis == 0 ? N % t != 0 : n % t != 0) return fail(TP_EDIVIS, "t=%d does not divide the scattered dim", t);
+  if (ring_gemm_fits(N, n, t, axis))
+    return fused_row_reduce(x, N, k / t, n, t, w, mode, axis, out, nullptr, TP_F32, nullptr, s);
+  if (partials == nullptr)
+    return fail(TP_EUNSUPPORTED, "chunks do not align with the fused kernel's 128 x 256 tiles and no partials were given");
+  if (tp_status st = row_gemm(x, N, k / t, n, t, w, partials, s)) return st;
+  RingArgs a = ring_args(mode == TP_OUT_RS ? RING_RS : RING_AR, t, N, n, axis, TP_F32, TP_F32);
+  for (int r = 0; r < t; ++r) { a.in[r] = partials[r]; a.out[r] = out[r]; }
+  return ring_collective(a, s);
+}
+
 tp_status tp_mlp_fwd(const uint16_t* x, int64_t N, int64_t h, int64_t F, int t, tp_act act, const uint16_t* w_in,
                      const uint16_t* w_down, uint16_t* z_ws, float* const* partials, tp_reduce mode, float* const* out,
                      void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (!valid_t(t)) return fail(TP_EINVAL, "t=%d outside 1..%d", t, TP_MAX_SHARDS);
-  if (x == nullptr || w_in == nullptr || w_down == nullptr || z_ws == nullptr || partials == nullptr)
-    return fail(TP_EINVAL, "null pointer");
+  if (x == nullptr || w_in == nullptr || w_down == nullptr || z_ws == nullptr) return fail(TP_EINVAL, "null pointer");
+  if (partials == nullptr && (mode == TP_OUT_PARTIALS || N % t != 0 || !ring_gemm_fits(N, h, t, 0)))
+    return fail(TP_EINVAL, "null partials: needed unless the fused row GEMM + reduction applies (N/t a multiple of 128)");
   if (!valid_act(act)) return fail(TP_EINVAL, "bad activation");
   if (mode < TP_OUT_PARTIALS || mode > TP_OUT_RS_AG) return fail(TP_EINVAL, "bad reduce mode");
   if (N <= 0 || h <= 0 || F <= 0) return fail(TP_EINVAL, "non-positive size");
@@ -144,6 +187,11 @@ tp_status tp_mlp_fwd(const uint16_t* x, int64_t N, int64_t h, int64_t F, int t, 
   if (mode != TP_OUT_PARTIALS && N % t) return fail(TP_EDIVIS, "t=%d does not divide the token count %lld", t, (long long)N);
   const int64_t f = F / t;
   if (tp_status st = column_gemm(x, N, h, f, t, act, w_in, z_ws, s)) return st;          // Z_r = act(X W_in[r])
+  if (mode != TP_OUT_PARTIALS && ring_gemm_fits(N, h, t, 0)) {
+    // U_r = Z_r W_down[r] and g (the collective) in one kernel; the partials never reach HBM
+    if (out == nullptr) return fail(TP_EINVAL, "null output array");
+    return fused_row_reduce(z_ws, N, f, h, t, w_down, mode, 0, out, nullptr, TP_F32, nullptr, s);
+  }
   if (tp_status st = row_gemm(z_ws, N, f, h, t, w_down, partials, s)) return st;         // U_r = Z_r W_down[r]
   return reduce_partials(partials, N, h, t, mode, out, nullptr, TP_F32, nullptr, s);     // g: the collective
 }
@@ -197,6 +245,13 @@ tp_status tp_sharded_matmul(int case_id, int strategy, const uint16_t* const* x,
       if (B % t) return fail(TP_EDIVIS, "t=%d does not divide B (AllReduce chunks)", t);
       const size_t slot = align256(size_t(B) * F * 4);
       const int64_t d = D / t;
+      if (ring_gemm_fits(B, F, t, 0)) {                 // local products and AllReduce in one kernel
+        RingGemmArgs rg;
+        std::memset(&rg, 0, sizeof(rg));
+        rg.t = t; rg.M = B; rg.N = F; rg.K = d; rg.lda = d; rg.ldb = F; rg.op = RING_AR; rg.out_dtype = c_dtype;
+        for (int i = 0; i < t; ++i) { rg.a[i] = x[i]; rg.b[i] = w[i] + i * d * F; rg.out[i] = c[i]; }
+        return ring_gemm(rg, s);
+      }
       GemmArgs g = gemm_args(t, B, F, d, d, F, EPI_F32);
       for (int i = 0; i < t; ++i) { g.a[i] = x[i]; g.b[i] = w[i] + i * d * F; g.c[i] = wsb + i * slot; }
       if (tp_status st = grouped_gemm(g, s)) return st;
@@ -214,6 +269,15 @@ tp_status tp_sharded_matmul(int case_id, int strategy, const uint16_t* const* x,
     GemmArgs g = gemm_args(t, B, F, d, d, F, EPI_F32);
     for (int i = 0; i < t; ++i) { g.a[i] = x[i]; g.b[i] = w[i]; g.c[i] = wsb + i * slot; }
     if (strategy == TP_CASE3_RS_F ? (F % t != 0) : (B % t != 0)) return fail(TP_EDIVIS, "t=%d does not divide the scattered dim", t);
+    const int axis = strategy == TP_CASE3_RS_F ? 1 : 0;
+    if (ring_gemm_fits(B, F, t, axis)) {                 // local products and the reduction in one kernel
+      RingGemmArgs rg;
+      std::memset(&rg, 0, sizeof(rg));
+      rg.t = t; rg.M = B; rg.N = F; rg.K = d; rg.lda = d; rg.ldb = F; rg.axis = axis; rg.out_dtype = c_dtype;
+      rg.op = strategy == TP_CASE3_ALLREDUCE ? RING_AR : RING_RS;
+      for (int i = 0; i < t; ++i) { rg.a[i] = x[i]; rg.b[i] = w[i]; rg.out[i] = c[i]; }
+      return ring_gemm(rg, s);
+    }
     if (tp_status st = grouped_gemm(g, s)) return st;
     RingArgs a = ring_args(strategy == TP_CASE3_ALLREDUCE ? RING_AR : RING_RS, t, B, F,
                            strategy == TP_CASE3_RS_F ? 1 : 0, TP_F32, c_dtype);
@@ -251,7 +315,7 @@ tp_status tp_layer_fwd(const uint16_t* x, const uint16_t* const* o, int64_t N, i
                        float* const* partials, float* const* y, void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (!valid_t(t)) return fail(TP_EINVAL, "t=%d outside 1..%d", t, TP_MAX_SHARDS);
-  if (!x || !o || !w_qkv || !w_o || !w_gu || !w_down || !qkv_out || !h1 || !h1_bf16 || !z_ws || !partials || !y)
+  if (!x || !o || !w_qkv || !w_o || !w_gu || !w_down || !qkv_out || !h1 || !h1_bf16 || !z_ws || !y)
     return fail(TP_EINVAL, "null pointer");
   if (N <= 0 || h <= 0 || F <= 0 || n_h <= 0 || n_kv <= 0 || d_h <= 0) return fail(TP_EINVAL, "non-positive size");
   if (n_h % t || n_h % n_kv || (t <= n_kv ? n_kv % t != 0 : t % n_kv != 0))
@@ -260,22 +324,33 @@ tp_status tp_layer_fwd(const uint16_t* x, const uint16_t* const* o, int64_t N, i
   const int64_t kv = t <= n_kv ? n_kv / t : 1;
   const int64_t qkv_w = (n_h / t + 2 * kv) * d_h;
   const int64_t o_w = int64_t(n_h) * d_h / t;
+  const bool need_partials = !ring_gemm_fits(N, h, t, 0);
+  if (need_partials && partials == nullptr) return fail(TP_EINVAL, "null partials (needed: N/t is not a multiple of 128)");
   for (int r = 0; r < t; ++r)
-    if (o[r] == nullptr || h1[r] == nullptr || partials[r] == nullptr || y[r] == nullptr)
+    if (o[r] == nullptr || h1[r] == nullptr || y[r] == nullptr || (need_partials && partials[r] == nullptr))
       return fail(TP_EINVAL, "null shard buffer %d", r);
   // 1. fused QKV projection, column-parallel on head boundaries (feeds the attention core)
   if (tp_status st = column_gemm(x, N, h, qkv_w, t, TP_ACT_NONE, w_qkv, qkv_out, s)) return st;
-  // 2. attention output projection, row-parallel: partials O_r W_o[r]
-  {
+  const bool fused = ring_gemm_fits(N, h, t, 0);
+  // 2-3. attention output projection (row-parallel) and g: AllReduce, with the residual add
+  //      h1 = X + attn and the bf16 copy for the MLP input
+  if (fused) {
+    RingGemmArgs rg;
+    std::memset(&rg, 0, sizeof(rg));
+    rg.t = t; rg.M = N; rg.N = h; rg.K = o_w; rg.lda = o_w; rg.ldb = h; rg.op = RING_AR; rg.out_dtype = TP_F32;
+    rg.resid = x; rg.resid_dtype = TP_BF16; rg.copy_bf16 = h1_bf16;
+    for (int r = 0; r < t; ++r) { rg.a[r] = o[r]; rg.b[r] = w_o + r * o_w * h; rg.out[r] = h1[r]; }
+    if (tp_status st = ring_gemm(rg, s)) return st;
+  } else {
     GemmArgs g = gemm_args(t, N, h, o_w, o_w, h, EPI_F32);
     for (int r = 0; r < t; ++r) { g.a[r] = o[r]; g.b[r] = w_o + r * o_w * h; g.c[r] = partials[r]; }
     if (tp_status st = grouped_gemm(g, s)) return st;
+    if (tp_status st = reduce_partials(partials, N, h, t, TP_OUT_AR, h1, x, TP_BF16, h1_bf16, s)) return st;
   }
-  // 3. g: AllReduce, fused with the residual add h1 = X + attn and the bf16 copy for the MLP input
-  if (tp_status st = reduce_partials(partials, N, h, t, TP_OUT_AR, h1, x, TP_BF16, h1_bf16, s)) return st;
-  // 4. SwiGLU MLP on bf16(h1), partials, then AllReduce fused with y = h1 + mlp
+  // 4. SwiGLU MLP on bf16(h1), then AllReduce with y = h1 + mlp
   const int64_t f = F / t;
   if (tp_status st = column_gemm(h1_bf16, N, h, f, t, TP_ACT_SWIGLU, w_gu, z_ws, s)) return st;
+  if (fused) return fused_row_reduce(z_ws, N, f, h, t, w_down, TP_OUT_AR, 0, y, h1[0], TP_F32, nullptr, s);
   if (tp_status st = row_gemm(z_ws, N, f, h, t, w_down, partials, s)) return st;
   return reduce_partials(partials, N, h, t, TP_OUT_AR, y, h1[0], TP_F32, nullptr, s);
 }

@@ -63,4 +63,24 @@ struct GemmArgs {
 };
 tp_status grouped_gemm(const GemmArgs& g, cudaStream_t s);
 
+// Row-parallel GEMM fused with its ring reduction: out = Reduce_s(a[s] . b[s]) over the t shards.
+// RING_RS: out[c] receives chunk c (rows for axis 0, columns for axis 1); RING_AR: every out[s]
+// receives the whole sum (+ resid), and copy_bf16 (optional) a bf16 copy.
+struct RingGemmArgs {
+  int t;
+  const uint16_t* a[TP_MAX_SHARDS];  // [M, K] row-major, row stride lda
+  const uint16_t* b[TP_MAX_SHARDS];  // [K, N] row-major, row stride ldb
+  void* out[TP_MAX_SHARDS];
+  int64_t M, N, K, lda, ldb;
+  RingOp op;                         // RING_RS or RING_AR
+  int axis;                          // RS chunk axis
+  tp_dtype out_dtype;
+  const void* resid;                 // RING_AR only, [M, N]
+  tp_dtype resid_dtype;
+  uint16_t* copy_bf16;               // RING_AR only, [M, N]
+};
+// True when every 128 x 256 output tile lies inside one chunk (the fused kernel's requirement).
+bool ring_gemm_fits(int64_t M, int64_t N, int t, int axis);
+tp_status ring_gemm(const RingGemmArgs& g, cudaStream_t s);
+
 }  // namespace tpx

@@ -1,22 +1,34 @@
-// Grouped bf16 GEMM on the 5th-generation tensor cores (tcgen05) with fused epilogues.
+// bf16 GEMMs on the 5th-generation tensor cores (tcgen05) with fused epilogues.
 //
-// Used for the column-parallel GEMM Z_r = act(X W_r) and the row-parallel GEMM U_r = Z_r W_r of the
-// tensor-parallel MLP ("张量并行与序列并行", §矩阵乘法的两种切法 and §MLP：先列后行，只通信一次), and for
-// the local products of the sharded-matmul cases ("Scaling Book 入门第 6 章", §6.2). All t shards
-// of one layer run in ONE persistent launch: the tile space is (shard, m-tile, n-tile).
+// Two persistent, warp-specialised kernels share one TMA -> shared memory -> tcgen05.mma -> TMEM
+// pipeline:
 //
-// Design (sm_100a):
-//   * persistent CTAs, one per SM, each looping over tiles (raster: bands of row-tiles swept across
-//     the n-tiles so that concurrently running CTAs share operand panels in L2);
-//   * warp 0, one lane: TMA producer. A [M,K] is K-major (box 64 x 128, 128-byte swizzle); B [K,N]
-//     is the weight as stored, [in, out] row-major, i.e. MN-major (boxes 64 x 64, 128-byte swizzle);
-//   * warp 1, one lane: tcgen05.mma issuer (M=128, N=256, K=16 per instruction, fp32 accumulator in
-//     TMEM). 4-stage shared-memory ring, two TMEM accumulators (2 x 256 columns) so the epilogue of
-//     one tile overlaps the main loop of the next;
-//   * warps 2..5: epilogue. tcgen05.ld 32 columns at a time, apply the activation in fp32, store.
-//     SwiGLU tiles carry 128 gate columns and the 128 up columns of the same F indices in one
-//     N=256 accumulator, so SiLU(gate)*up is formed in registers without another pass.
-//   * every mbarrier wait is bounded; on expiry the kernel records the site in the status word,
+//  gemm_tcgen05_kernel: grouped GEMM C_g = epi(A_g B_g). It serves the column-parallel GEMM
+//    Z_r = act(X W_r), the row-parallel GEMM U_r = Z_r W_r when the partials themselves are wanted
+//    ("张量并行与序列并行", §矩阵乘法的两种切法 and §MLP：先列后行，只通信一次), and the local
+//    products of the sharded-matmul cases ("Scaling Book 入门第 6 章", §6.2). All t shards of one
+//    layer run in ONE launch over the tile space (shard, m-tile, n-tile).
+//
+//  gemm_ring_kernel: the row-parallel GEMM fused with its collective, the one-GPU form of the
+//    pages' collective matmul ("Scaling Book 入门第 6 章", §6.6; "张量并行与序列并行",
+//    §把通信藏到计算后面). For each output tile it computes the t shards' partial tiles
+//    U_s = A_s B_s one after another IN RING ORDER (s = c+1, c+2, ..., c for the tile's chunk c) into
+//    alternating TMEM accumulators. The epilogue adds them into an fp32 running sum in registers, one
+//    binary32 add per shard, which is exactly the ReduceScatter's summation order. It then writes the
+//    tile once: to shard c's output (ReduceScatter) or to all t outputs (AllReduce = ReduceScatter
+//    followed by AllGather), optionally adding a residual and writing a bf16 copy. The fp32 partials
+//    never reach HBM. Each U_s tile comes from the same instruction sequence as
+//    gemm_tcgen05_kernel's, so the results are bit-identical to the unfused GEMM followed by the
+//    ring kernel.
+//
+// Pipeline (sm_100a):
+//   * warp 0, one lane: TMA producer. A [M,K] is K-major (box 64 x 128, 128-byte swizzle); B [K,N] is
+//     the weight as stored, [in, out] row-major, i.e. MN-major (four 64 x 64 boxes, 128-byte swizzle);
+//   * warp 1, one lane: tcgen05.mma issuer (M=128, N=256, K=16 per instruction, fp32 in TMEM);
+//     4-stage shared-memory ring; two TMEM accumulators of 256 columns, so the epilogue of one unit
+//     overlaps the main loop of the next;
+//   * the remaining warps: epilogue (tcgen05.ld 32 columns at a time);
+//   * every mbarrier wait is bounded: on expiry the kernel records the site in the status word,
 //     raises a shared abort flag, drains its in-flight copies and MMAs and frees TMEM.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -35,45 +47,189 @@ constexpr int BM = 128;
 constexpr int BN = 256;                  // MMA N (output tile width; 128 for SwiGLU)
 constexpr int BK = 64;                   // one 128-byte swizzle atom of bf16
 constexpr int STAGES = 4;
-constexpr int THREADS = 192;
 constexpr uint32_t A_STAGE = BM * BK * 2;        // 16 KiB
 constexpr uint32_t B_STAGE = BN * BK * 2;        // 32 KiB
 constexpr uint32_t B_BOX = 64 * BK * 2;          // one 64(N) x 64(K) box, 8 KiB
 constexpr uint32_t TMEM_COLS = 512;              // two 128 x 256 fp32 accumulators
 constexpr int RASTER_BAND = 16;                  // row-tiles per raster band
-constexpr size_t SMEM_BYTES = 1024 + STAGES * (A_STAGE + B_STAGE) + 256;
 constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, /*a_mn=*/false, /*b_mn=*/true);
 
-struct GemmParams {
-  CUtensorMap ta[TP_MAX_SHARDS];    // A views
-  CUtensorMap tb[TP_MAX_SHARDS];    // B views (the gate half for SwiGLU)
-  CUtensorMap tb2[TP_MAX_SHARDS];   // up-half views (SwiGLU only)
-  void* c[TP_MAX_SHARDS];
-  int M, N, K;                      // N = output columns
-  int groups, tiles_m, tiles_n, row_tiles, num_tiles, num_kb;
+constexpr int GEMM_THREADS = 192;                // producer, MMA, 4 epilogue warps
+constexpr int RING_THREADS = 320;                // producer, MMA, 8 epilogue warps
+constexpr uint32_t STAGING_PER_WARP = 32 * 128;  // 32 rows x 128 bytes
+constexpr size_t GEMM_SMEM = 1024 + STAGES * (A_STAGE + B_STAGE) + 256;
+// CTA-pair (cta_group::2) variant: a 256 x 256 tile per pair, each CTA holding 128 rows of A and
+// 128 of B's columns per stage, so a 6-stage ring fits.
+constexpr int PAIR_STAGES = 6;
+constexpr uint32_t PAIR_A_STAGE = 128 * BK * 2;  // 16 KiB
+constexpr uint32_t PAIR_B_STAGE = 128 * BK * 2;  // 16 KiB: two 64-wide boxes
+constexpr size_t PAIR_SMEM = 1024 + PAIR_STAGES * (PAIR_A_STAGE + PAIR_B_STAGE) + 256;
+constexpr uint32_t IDESC_PAIR = idesc_bf16_f32(2 * BM, BN, /*a_mn=*/false, /*b_mn=*/true);
+constexpr size_t RING_SMEM = 1024 + STAGES * (A_STAGE + B_STAGE) + 8 * STAGING_PER_WARP + 256;
+
+// ------------------------------------------------------------------ shared pipeline pieces
+struct Ring {
+  int stage = 0;
+  uint32_t phase = 0;
+  __device__ __forceinline__ void advance() {
+    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+  }
+};
+
+struct Ctl {
+  uint8_t* sA;
+  uint8_t* sB;
+  uint32_t full0, empty0, accf0, acce0, drain;
+  volatile uint32_t* abort_flag;
   uint32_t* status;
   unsigned long long budget;
 };
 
-struct Tile {
-  int g, m0, n0;
-};
+__device__ __forceinline__ bool wait_or_abort(const Ctl& c, uint32_t bar, uint32_t parity, uint32_t site) {
+  if (mbar_wait_bounded(bar, parity, c.budget, c.abort_flag)) return true;
+  if (!*c.abort_flag) record_timeout(c.status, site);
+  *c.abort_flag = 1u;
+  return false;
+}
 
-// Tile index -> (shard, m0, n0). Row-tiles of all shards form one sequence (shard-major); it is cut
-// into bands of RASTER_BAND row-tiles and each band is swept across all n-tiles, row-tile fastest.
-__device__ __forceinline__ Tile decode_tile(const GemmParams& p, int tile, int tile_n_cols) {
-  const int band_tiles = RASTER_BAND * p.tiles_n;
+// Lays out barriers and the TMEM slot after the operand stages (and the staging area, if any).
+__device__ __forceinline__ Ctl setup_ctl(uint8_t* smem, uint32_t extra_bytes, uint32_t*& tmem_slot, uint32_t* status,
+                                         unsigned long long budget) {
+  Ctl c;
+  c.sA = smem;
+  c.sB = smem + STAGES * A_STAGE;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(c.sB + STAGES * B_STAGE + extra_bytes);
+  c.full0 = smem_u32(bars);
+  c.empty0 = c.full0 + 8 * STAGES;
+  c.accf0 = c.empty0 + 8 * STAGES;
+  c.acce0 = c.accf0 + 16;
+  c.drain = c.acce0 + 16;
+  tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+  c.abort_flag = tmem_slot + 1;
+  c.status = status;
+  c.budget = budget;
+  return c;
+}
+
+__device__ __forceinline__ void init_barriers(const Ctl& c, uint32_t epilogue_warps) {
+  for (int s = 0; s < STAGES; ++s) {
+    mbar_init(c.full0 + 8 * s, 1);
+    mbar_init(c.empty0 + 8 * s, 1);
+  }
+  for (int a = 0; a < 2; ++a) {
+    mbar_init(c.accf0 + 8 * a, 1);
+    mbar_init(c.acce0 + 8 * a, epilogue_warps);   // one arrive per epilogue warp
+  }
+  mbar_init(c.drain, 1);
+  *c.abort_flag = 0u;
+  fence_mbar_init();
+}
+
+// Producer: the num_kb k-blocks of one unit. B is four 64-wide boxes of `b` at n0 (b2 == nullptr),
+// or two boxes of `b` and two of `b2`, both at n0 (SwiGLU: gate and up halves).
+__device__ __forceinline__ bool produce_unit(const Ctl& c, Ring& r, const CUtensorMap* a, const CUtensorMap* b,
+                                             const CUtensorMap* b2, int m0, int n0, int num_kb, int* last_phase,
+                                             bool* issued) {
+  for (int kb = 0; kb < num_kb; ++kb) {
+    if (!wait_or_abort(c, c.empty0 + 8 * r.stage, r.phase ^ 1u, WAIT_PRODUCER_EMPTY)) return false;
+    const uint32_t fb = c.full0 + 8 * r.stage;
+    mbar_arrive_expect_tx(fb, A_STAGE + B_STAGE);
+    const uint32_t a_dst = smem_u32(c.sA + r.stage * A_STAGE);
+    const uint32_t b_dst = smem_u32(c.sB + r.stage * B_STAGE);
+    const int k0 = kb * BK;
+    tma_load_2d(a_dst, a, k0, m0, fb);
+    if (b2 != nullptr) {
+      tma_load_2d(b_dst + 0 * B_BOX, b, n0, k0, fb);
+      tma_load_2d(b_dst + 1 * B_BOX, b, n0 + 64, k0, fb);
+      tma_load_2d(b_dst + 2 * B_BOX, b2, n0, k0, fb);
+      tma_load_2d(b_dst + 3 * B_BOX, b2, n0 + 64, k0, fb);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) tma_load_2d(b_dst + j * B_BOX, b, n0 + 64 * j, k0, fb);
+    }
+    issued[r.stage] = true;
+    last_phase[r.stage] = static_cast<int>(r.phase);
+    r.advance();
+  }
+  return true;
+}
+
+// MMA issuer: accumulate one unit's num_kb k-blocks into d_tmem (the first one overwrites).
+__device__ __forceinline__ bool mma_unit(const Ctl& c, Ring& r, uint32_t d_tmem, int num_kb, bool& mma_issued) {
+  for (int kb = 0; kb < num_kb; ++kb) {
+    if (!wait_or_abort(c, c.full0 + 8 * r.stage, r.phase, WAIT_MMA_FULL)) return false;
+    tc_fence_after();
+    const uint32_t a_base = smem_u32(c.sA + r.stage * A_STAGE);
+    const uint32_t b_base = smem_u32(c.sB + r.stage * B_STAGE);
+#pragma unroll
+    for (int k = 0; k < BK / 16; ++k) {
+      // K-major A: advance 16 elements = 32 bytes inside the swizzle atom.
+      const uint64_t ad = smem_desc_sw128(a_base + 32u * k, 16u, 1024u);
+      // MN-major B: advance 16 K rows = two 8-row groups of 1 KiB; 64-wide N blocks 8 KiB apart.
+      const uint64_t bd = smem_desc_sw128(b_base + 2048u * k, B_BOX, 1024u);
+      umma_bf16(d_tmem, ad, bd, IDESC, (kb | k) != 0 ? 1u : 0u);
+    }
+    mma_issued = true;
+    umma_commit(c.empty0 + 8 * r.stage);   // frees the stage once these MMAs have read it
+    r.advance();
+  }
+  return true;
+}
+
+// After all roles left their loops: if the kernel aborted, wait (bounded) for the copies and MMAs
+// still in flight, then free TMEM. Called by every thread.
+__device__ __forceinline__ void teardown(const Ctl& c, int warp, int lane, const int* last_phase, const bool* issued,
+                                         bool mma_issued, uint32_t tmem_base) {
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (*c.abort_flag != 0u) {
+    const unsigned long long drain_budget = 4000000000ull;
+    if (warp == 0 && lane == 0) {
+      for (int s = 0; s < STAGES; ++s)
+        if (issued[s] && !mbar_wait_bounded(c.full0 + 8 * s, static_cast<uint32_t>(last_phase[s]), drain_budget, nullptr))
+          record_timeout(c.status, WAIT_TEARDOWN);
+    }
+    if (warp == 1 && lane == 0 && mma_issued) {
+      umma_commit(c.drain);
+      if (!mbar_wait_bounded(c.drain, 0, drain_budget, nullptr)) record_timeout(c.status, WAIT_TEARDOWN);
+    }
+  }
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
+}
+
+// Tile index -> (row-tile, n-tile). Row-tiles form one sequence; it is cut into bands of
+// RASTER_BAND row-tiles and each band is swept across all n-tiles, row-tile fastest.
+__device__ __forceinline__ void raster(int tile, int row_tiles, int tiles_n, int& rt, int& nt) {
+  const int band_tiles = RASTER_BAND * tiles_n;
   const int band = tile / band_tiles;
   const int first = band * RASTER_BAND;
-  const int in_band = min(RASTER_BAND, p.row_tiles - first);
+  const int in_band = min(RASTER_BAND, row_tiles - first);
   const int local = tile - band * band_tiles;
-  const int rt = first + local % in_band;
-  const int nt = local / in_band;
-  Tile t;
-  t.g = rt / p.tiles_m;
-  t.m0 = (rt - t.g * p.tiles_m) * BM;
-  t.n0 = nt * tile_n_cols;
-  return t;
+  rt = first + local % in_band;
+  nt = local / in_band;
+}
+
+// Fused-kernel tile order: chunk by chunk, so that every running tile streams the same shard's
+// operands at about the same time (all tiles of a chunk follow the same ring order). Axis 0: the
+// chunk's row-tiles fastest, then its n-tiles. Axis 1: all row-tiles fastest, then the chunk's n-tiles.
+__device__ __forceinline__ void raster_by_chunk(int tile, int tiles_m, int tiles_n, int axis, int chunk_tiles, int& rt,
+                                                int& nt) {
+  if (axis == 0) {
+    const int per_chunk = chunk_tiles * tiles_n;           // chunk_tiles row-tiles per chunk
+    const int c = tile / per_chunk;
+    const int local = tile - c * per_chunk;
+    rt = c * chunk_tiles + local % chunk_tiles;
+    nt = local / chunk_tiles;
+  } else {
+    const int per_chunk = tiles_m * chunk_tiles;           // chunk_tiles n-tiles per chunk
+    const int c = tile / per_chunk;
+    const int local = tile - c * per_chunk;
+    rt = local % tiles_m;
+    nt = c * chunk_tiles + local / tiles_m;
+  }
 }
 
 __device__ __forceinline__ float gelu_erf(float x) { return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f)); }
@@ -86,6 +242,18 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
   return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(lo))) |
          (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(hi))) << 16);
 }
+
+// ------------------------------------------------------------------ grouped GEMM
+struct GemmParams {
+  CUtensorMap ta[TP_MAX_SHARDS];    // A views
+  CUtensorMap tb[TP_MAX_SHARDS];    // B views (the gate half for SwiGLU)
+  CUtensorMap tb2[TP_MAX_SHARDS];   // up-half views (SwiGLU only)
+  void* c[TP_MAX_SHARDS];
+  int M, N, K;                      // N = output columns
+  int groups, tiles_m, tiles_n, row_tiles, num_tiles, num_kb;
+  uint32_t* status;
+  unsigned long long budget;
+};
 
 // Store 32 consecutive output columns [col0, col0+32) of one row.
 template <int EPI>
@@ -116,40 +284,18 @@ __device__ __forceinline__ void store_row_chunk(void* cbase, int N, int row, int
 }
 
 template <int EPI>
-__global__ void __launch_bounds__(THREADS, 1) gemm_tcgen05_kernel(const __grid_constant__ GemmParams p) {
+__global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tcgen05_kernel(const __grid_constant__ GemmParams p) {
   constexpr bool SWIGLU = EPI == EPI_SWIGLU;
   constexpr int TILE_N = SWIGLU ? BN / 2 : BN;   // output columns per tile
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sA = smem;
-  uint8_t* sB = smem + STAGES * A_STAGE;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * B_STAGE);
-  // bars: full[STAGES], empty[STAGES], acc_full[2], acc_empty[2], drain
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
-  volatile uint32_t* abort_flag = tmem_slot + 1;
-
+  uint32_t* tmem_slot;
+  const Ctl c = setup_ctl(smem, 0, tmem_slot, p.status, p.budget);
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  const uint32_t full0 = smem_u32(bars);
-  const uint32_t empty0 = full0 + 8 * STAGES;
-  const uint32_t accf0 = empty0 + 8 * STAGES;
-  const uint32_t acce0 = accf0 + 16;
-  const uint32_t drain = acce0 + 16;
 
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(full0 + 8 * s, 1);
-      mbar_init(empty0 + 8 * s, 1);
-    }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(accf0 + 8 * a, 1);
-      mbar_init(acce0 + 8 * a, 4);   // one arrive per epilogue warp
-    }
-    mbar_init(drain, 1);
-    *abort_flag = 0u;
-    fence_mbar_init();
-  }
+  if (threadIdx.x == 0) init_barriers(c, 4);
   if (warp == 0 && lane == 0) {
     for (int g = 0; g < p.groups; ++g) {
       prefetch_tmap(&p.ta[g]);
@@ -166,7 +312,6 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tcgen05_kernel(const __grid_c
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  // producer bookkeeping, used again at teardown
   int last_phase[STAGES];
   bool issued[STAGES];
 #pragma unroll
@@ -175,79 +320,27 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tcgen05_kernel(const __grid_c
 
   if (warp == 0) {
     if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
+      Ring r;
       for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
-        const Tile tl = decode_tile(p, tile, TILE_N);
-        bool ok = true;
-        for (int kb = 0; kb < p.num_kb; ++kb) {
-          if (!mbar_wait_bounded(empty0 + 8 * stage, phase ^ 1u, p.budget, abort_flag)) {
-            if (!*abort_flag) record_timeout(p.status, WAIT_PRODUCER_EMPTY);
-            *abort_flag = 1u;
-            ok = false;
-            break;
-          }
-          const uint32_t fb = full0 + 8 * stage;
-          mbar_arrive_expect_tx(fb, A_STAGE + B_STAGE);
-          const uint32_t a_dst = smem_u32(sA + stage * A_STAGE);
-          const uint32_t b_dst = smem_u32(sB + stage * B_STAGE);
-          const int k0 = kb * BK;
-          tma_load_2d(a_dst, &p.ta[tl.g], k0, tl.m0, fb);
-          if constexpr (SWIGLU) {
-            tma_load_2d(b_dst + 0 * B_BOX, &p.tb[tl.g], tl.n0, k0, fb);
-            tma_load_2d(b_dst + 1 * B_BOX, &p.tb[tl.g], tl.n0 + 64, k0, fb);
-            tma_load_2d(b_dst + 2 * B_BOX, &p.tb2[tl.g], tl.n0, k0, fb);
-            tma_load_2d(b_dst + 3 * B_BOX, &p.tb2[tl.g], tl.n0 + 64, k0, fb);
-          } else {
-#pragma unroll
-            for (int j = 0; j < 4; ++j) tma_load_2d(b_dst + j * B_BOX, &p.tb[tl.g], tl.n0 + 64 * j, k0, fb);
-          }
-          issued[stage] = true;
-          last_phase[stage] = static_cast<int>(phase);
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-        }
-        if (!ok) break;
+        int rt, nt;
+        raster(tile, p.row_tiles, p.tiles_n, rt, nt);
+        const int g = rt / p.tiles_m;
+        const int m0 = (rt - g * p.tiles_m) * BM;
+        if (!produce_unit(c, r, &p.ta[g], &p.tb[g], SWIGLU ? &p.tb2[g] : nullptr, m0, nt * TILE_N, p.num_kb,
+                          last_phase, issued))
+          break;
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
+      Ring r;
       int acc = 0;
       uint32_t acc_phase = 0;
       for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
-        bool ok = mbar_wait_bounded(acce0 + 8 * acc, acc_phase ^ 1u, p.budget, abort_flag);
-        if (!ok) {
-          if (!*abort_flag) record_timeout(p.status, WAIT_MMA_ACC_EMPTY);
-          *abort_flag = 1u;
-          break;
-        }
+        if (!wait_or_abort(c, c.acce0 + 8 * acc, acc_phase ^ 1u, WAIT_MMA_ACC_EMPTY)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
-        for (int kb = 0; kb < p.num_kb; ++kb) {
-          if (!mbar_wait_bounded(full0 + 8 * stage, phase, p.budget, abort_flag)) {
-            if (!*abort_flag) record_timeout(p.status, WAIT_MMA_FULL);
-            *abort_flag = 1u;
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t a_base = smem_u32(sA + stage * A_STAGE);
-          const uint32_t b_base = smem_u32(sB + stage * B_STAGE);
-#pragma unroll
-          for (int k = 0; k < BK / 16; ++k) {
-            // K-major A: advance 16 elements = 32 bytes inside the swizzle atom.
-            const uint64_t ad = smem_desc_sw128(a_base + 32u * k, 16u, 1024u);
-            // MN-major B: advance 16 K rows = two 8-row groups of 1 KiB; 64-wide N blocks 8 KiB apart.
-            const uint64_t bd = smem_desc_sw128(b_base + 2048u * k, B_BOX, 1024u);
-            umma_bf16(d_tmem, ad, bd, IDESC, (kb | k) != 0 ? 1u : 0u);
-          }
-          mma_issued = true;
-          umma_commit(empty0 + 8 * stage);   // frees the stage once these MMAs have read it
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-        }
-        if (!ok) break;
-        umma_commit(accf0 + 8 * acc);        // accumulator complete
+        if (!mma_unit(c, r, tmem_base + static_cast<uint32_t>(acc * BN), p.num_kb, mma_issued)) break;
+        umma_commit(c.accf0 + 8 * acc);   // accumulator complete
         if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
       }
     }
@@ -257,51 +350,424 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tcgen05_kernel(const __grid_c
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
-      const Tile tl = decode_tile(p, tile, TILE_N);
-      if (!mbar_wait_bounded(accf0 + 8 * acc, acc_phase, p.budget, abort_flag)) {
-        if (!*abort_flag) record_timeout(p.status, WAIT_EPI_ACC_FULL);
-        *abort_flag = 1u;
-        break;
-      }
+      int rt, nt;
+      raster(tile, p.row_tiles, p.tiles_n, rt, nt);
+      const int g = rt / p.tiles_m;
+      const int m0 = (rt - g * p.tiles_m) * BM;
+      const int n0 = nt * TILE_N;
+      if (!wait_or_abort(c, c.accf0 + 8 * acc, acc_phase, WAIT_EPI_ACC_FULL)) break;
       tc_fence_after();
-      const int row = tl.m0 + quad * 32 + lane;
+      const int row = m0 + quad * 32 + lane;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * BN);
-      void* cbase = p.c[tl.g];
+      void* cbase = p.c[g];
 #pragma unroll 1
       for (int ch = 0; ch < TILE_N / 32; ++ch) {
         uint32_t v[32], u[32];
         tmem_ld32(t_row + ch * 32, v);
         if constexpr (SWIGLU) tmem_ld32(t_row + 128 + ch * 32, u);
         tmem_ld_wait();
-        const int col0 = tl.n0 + ch * 32;
+        const int col0 = n0 + ch * 32;
         if (row < p.M && col0 < p.N) store_row_chunk<EPI>(cbase, p.N, row, col0, v, u);
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(acce0 + 8 * acc);
+      if (lane == 0) mbar_arrive(c.acce0 + 8 * acc);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+  }
+  teardown(c, warp, lane, last_phase, issued, mma_issued, tmem_base);
+}
+
+// ------------------------------------------------------------------ CTA-pair grouped GEMM
+// Same computation as gemm_tcgen05_kernel, on 256-row tiles shared by the two CTAs of a cluster.
+// Each CTA loads its 128 rows of A and its half of B's 256 columns (SwiGLU: CTA 0 the gate half, CTA 1
+// the up half) into its own shared memory. The copies of both CTAs count on the leader's barrier.
+// The leader's single MMA thread issues tcgen05.mma.cta_group::2 (M=256, N=256). Each CTA's TMEM
+// receives its own 128 rows, and each CTA's epilogue stores them.
+template <int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
+    gemm_pair_kernel(const __grid_constant__ GemmParams p) {
+  constexpr bool SWIGLU = EPI == EPI_SWIGLU;
+  constexpr int TILE_N = SWIGLU ? BN / 2 : BN;
+  constexpr int TILE_M = 2 * BM;
+
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + PAIR_STAGES * PAIR_A_STAGE;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + PAIR_STAGES * PAIR_B_STAGE);
+  const uint32_t full0 = smem_u32(bars);
+  const uint32_t empty0 = full0 + 8 * PAIR_STAGES;
+  const uint32_t accf0 = empty0 + 8 * PAIR_STAGES;
+  const uint32_t acce0 = accf0 + 16;
+  const uint32_t drain = acce0 + 16;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * PAIR_STAGES + 5);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < PAIR_STAGES; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(accf0 + 8 * a, 1);
+      mbar_init(acce0 + 8 * a, 8);   // 4 epilogue warps in each CTA of the pair
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0u;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    for (int g = 0; g < p.groups; ++g) {
+      prefetch_tmap(&p.ta[g]);
+      prefetch_tmap(rank == 1 && SWIGLU ? &p.tb2[g] : &p.tb[g]);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();   // barriers of both CTAs initialised, TMEM allocated
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const uint32_t full0_leader = mapa_shared(full0, 0);
+  const uint32_t acce0_leader = mapa_shared(acce0, 0);
+  const int pair = blockIdx.x >> 1;
+  const int pairs = gridDim.x >> 1;
+  const int tiles_m = (p.M + TILE_M - 1) / TILE_M;
+  const int row_tiles = p.groups * tiles_m;
+  const int num_tiles = row_tiles * p.tiles_n;
+  const unsigned long long budget = p.budget;
+  bool mma_issued = false;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = pair; ok && tile < num_tiles; tile += pairs) {
+        int rt, nt;
+        raster(tile, row_tiles, p.tiles_n, rt, nt);
+        const int g = rt / tiles_m;
+        const int m0 = (rt - g * tiles_m) * TILE_M + static_cast<int>(rank) * BM;
+        const int n0 = nt * TILE_N;
+        const CUtensorMap* tb = SWIGLU ? (rank == 0 ? &p.tb[g] : &p.tb2[g]) : &p.tb[g];
+        const int nb = SWIGLU ? n0 : n0 + static_cast<int>(rank) * 128;
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!mbar_wait_bounded(empty0 + 8 * stage, phase ^ 1u, budget, abort_flag)) {
+            if (!*abort_flag) record_timeout(p.status, WAIT_PRODUCER_EMPTY);
+            *abort_flag = 1u;
+            ok = false;
+            break;
+          }
+          if (leader) mbar_arrive_expect_tx(full0 + 8 * stage, 2 * (PAIR_A_STAGE + PAIR_B_STAGE));
+          const uint32_t fb = full0_leader + 8 * stage;
+          const uint32_t a_dst = smem_u32(sA + stage * PAIR_A_STAGE);
+          const uint32_t b_dst = smem_u32(sB + stage * PAIR_B_STAGE);
+          const int k0 = kb * BK;
+          tma_load_2d_pair(a_dst, &p.ta[g], k0, m0, fb);
+          tma_load_2d_pair(b_dst, tb, nb, k0, fb);
+          tma_load_2d_pair(b_dst + B_BOX, tb, nb + 64, k0, fb);
+          if (++stage == PAIR_STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = pair; ok && tile < num_tiles; tile += pairs) {
+        // the epilogues of BOTH CTAs release an accumulator on the leader's barrier
+        bool got = mbar_try_wait_cluster(acce0 + 8 * acc, acc_phase ^ 1u);
+        if (!got) {
+          const long long t0 = clock64();
+          while (!(got = mbar_try_wait_cluster(acce0 + 8 * acc, acc_phase ^ 1u))) {
+            if (*abort_flag || static_cast<unsigned long long>(clock64() - t0) > budget) break;
+          }
+        }
+        if (!got) {
+          if (!*abort_flag) record_timeout(p.status, WAIT_MMA_ACC_EMPTY);
+          *abort_flag = 1u;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!mbar_wait_bounded(full0 + 8 * stage, phase, budget, abort_flag)) {
+            if (!*abort_flag) record_timeout(p.status, WAIT_MMA_FULL);
+            *abort_flag = 1u;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(sA + stage * PAIR_A_STAGE);
+          const uint32_t b_base = smem_u32(sB + stage * PAIR_B_STAGE);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint64_t ad = smem_desc_sw128(a_base + 32u * k, 16u, 1024u);
+            const uint64_t bd = smem_desc_sw128(b_base + 2048u * k, B_BOX, 1024u);
+            umma_bf16_pair(d_tmem, ad, bd, IDESC_PAIR, (kb | k) != 0 ? 1u : 0u);
+          }
+          mma_issued = true;
+          umma_commit_pair_mc(empty0 + 8 * stage, 0x3);   // frees the stage in both CTAs
+          if (++stage == PAIR_STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit_pair_mc(accf0 + 8 * acc, 0x3);          // both halves of the accumulator ready
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      }
+    }
+  } else {
+    const int quad = warp & 3;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = pair; tile < num_tiles; tile += pairs) {
+      int rt, nt;
+      raster(tile, row_tiles, p.tiles_n, rt, nt);
+      const int g = rt / tiles_m;
+      const int m0 = (rt - g * tiles_m) * TILE_M + static_cast<int>(rank) * BM;
+      const int n0 = nt * TILE_N;
+      if (!mbar_wait_bounded(accf0 + 8 * acc, acc_phase, budget, abort_flag)) {
+        if (!*abort_flag) record_timeout(p.status, WAIT_EPI_ACC_FULL);
+        *abort_flag = 1u;
+        break;
+      }
+      tc_fence_after();
+      const int row = m0 + quad * 32 + lane;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * BN);
+      void* cbase = p.c[g];
+#pragma unroll 1
+      for (int ch = 0; ch < TILE_N / 32; ++ch) {
+        uint32_t v[32], u[32];
+        tmem_ld32(t_row + ch * 32, v);
+        if constexpr (SWIGLU) tmem_ld32(t_row + 128 + ch * 32, u);
+        tmem_ld_wait();
+        const int col0 = n0 + ch * 32;
+        if (row < p.M && col0 < p.N) store_row_chunk<EPI>(cbase, p.N, row, col0, v, u);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acce0_leader + 8 * acc);
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
   }
 
-  // ---- teardown: drain in-flight TMA and MMA work before TMEM is released -------------------
+  // teardown: all pair MMAs complete (they read both CTAs' shared memory and write both TMEMs),
+  // then both CTAs meet before either releases TMEM or exits.
   __syncwarp();
   tc_fence_before();
   __syncthreads();
-  if (*abort_flag != 0u) {
-    const unsigned long long drain_budget = 4000000000ull;
-    if (warp == 0 && lane == 0) {
-      for (int s = 0; s < STAGES; ++s)
-        if (issued[s] && !mbar_wait_bounded(full0 + 8 * s, static_cast<uint32_t>(last_phase[s]), drain_budget, nullptr))
-          record_timeout(p.status, WAIT_TEARDOWN);
-    }
-    if (warp == 1 && lane == 0 && mma_issued) {
-      umma_commit(drain);
-      if (!mbar_wait_bounded(drain, 0, drain_budget, nullptr)) record_timeout(p.status, WAIT_TEARDOWN);
+  if (warp == 1 && lane == 0 && leader && mma_issued) {
+    umma_commit_pair(drain);
+    if (!mbar_wait_bounded(drain, 0, 4000000000ull, nullptr)) record_timeout(p.status, WAIT_TEARDOWN);
+  }
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_pair(tmem_base, TMEM_COLS);
+}
+
+// ------------------------------------------------------------------ fused row GEMM + ring reduction
+struct RingGemmParams {
+  CUtensorMap ta[TP_MAX_SHARDS];    // A_s [M, K] (K-major)
+  CUtensorMap tb[TP_MAX_SHARDS];    // B_s [K, N] (MN-major)
+  void* out[TP_MAX_SHARDS];
+  const void* resid;                // AllReduce only: added after the ring sum (f32 or bf16 [M, N])
+  uint16_t* copy_bf16;              // AllReduce only: bf16 copy of the result [M, N]
+  int M, N, t;
+  int tiles_m, tiles_n, num_tiles, num_kb;
+  int axis;                         // chunk axis of the reduction
+  int chunk;                        // rows (axis 0) or columns (axis 1) per chunk
+  int chunk_tiles;                  // row-tiles (axis 0) or n-tiles (axis 1) per chunk
+  int resid_bf16;
+  uint32_t* status;
+  unsigned long long budget;
+};
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, float a, float b, float c, float d) {
+  asm volatile("st.shared.v4.f32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
+}
+__device__ __forceinline__ float4 ld_shared_v4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr) : "memory");
+  return v;
+}
+
+// Writes a 32 x 32 fp32 block held one row per lane (lane i: row row0+i, columns col0..col0+31)
+// with coalesced global stores. The block passes through the warp's 4 KiB staging buffer, with its
+// 16-byte chunks XOR-swizzled by row so both the row-wise writes and the column-wise reads are free
+// of bank conflicts. Each store instruction then covers four rows x 128 contiguous bytes (64 for bf16).
+template <bool OUT_BF16, bool AR>
+__device__ __forceinline__ void store_block32(const RingGemmParams& p, uint32_t stg, int lane, const float (&v)[32],
+                                              int row0, int col0, int c) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    st_shared_v4(stg + lane * 128 + ((j ^ (lane & 7)) << 4), v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+  __syncwarp();
+  const int sub = lane & 7;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int r = 4 * k + (lane >> 3);
+    float4 x = ld_shared_v4(stg + r * 128 + ((sub ^ (r & 7)) << 4));
+    const int row = row0 + r;
+    const int col = col0 + 4 * sub;
+    if (row < p.M && col < p.N) {
+      const int64_t e = static_cast<int64_t>(row) * p.N + col;
+      if constexpr (AR) {
+        if (p.resid != nullptr) {
+          float4 q;
+          if (p.resid_bf16) {
+            const uint2 w = *reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(p.resid) + e);
+            q = make_float4(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xFFFF0000u), __uint_as_float(w.y << 16),
+                            __uint_as_float(w.y & 0xFFFF0000u));
+          } else {
+            q = *reinterpret_cast<const float4*>(static_cast<const float*>(p.resid) + e);
+          }
+          x.x = __fadd_rn(x.x, q.x); x.y = __fadd_rn(x.y, q.y); x.z = __fadd_rn(x.z, q.z); x.w = __fadd_rn(x.w, q.w);
+        }
+        for (int s = 0; s < p.t; ++s) {
+          if constexpr (OUT_BF16)
+            *reinterpret_cast<uint2*>(static_cast<uint16_t*>(p.out[s]) + e) = make_uint2(pack2(x.x, x.y), pack2(x.z, x.w));
+          else
+            *reinterpret_cast<float4*>(static_cast<float*>(p.out[s]) + e) = x;
+        }
+        if (p.copy_bf16 != nullptr)
+          *reinterpret_cast<uint2*>(p.copy_bf16 + e) = make_uint2(pack2(x.x, x.y), pack2(x.z, x.w));
+      } else {
+        // ReduceScatter: chunk c lands in shard c's output, at its place inside the chunk
+        const int64_t o = p.axis == 0 ? static_cast<int64_t>(row - c * p.chunk) * p.N + col
+                                      : static_cast<int64_t>(row) * p.chunk + (col - c * p.chunk);
+        if constexpr (OUT_BF16)
+          *reinterpret_cast<uint2*>(static_cast<uint16_t*>(p.out[c]) + o) = make_uint2(pack2(x.x, x.y), pack2(x.z, x.w));
+        else
+          *reinterpret_cast<float4*>(static_cast<float*>(p.out[c]) + o) = x;
+      }
     }
   }
+  __syncwarp();
+}
+
+template <bool OUT_BF16, bool AR>
+__global__ void __launch_bounds__(RING_THREADS, 1) gemm_ring_kernel(const __grid_constant__ RingGemmParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint32_t* tmem_slot;
+  const Ctl c = setup_ctl(smem, 8 * STAGING_PER_WARP, tmem_slot, p.status, p.budget);
+  const uint32_t staging0 = smem_u32(smem + STAGES * (A_STAGE + B_STAGE));
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const int t = p.t;
+
+  if (threadIdx.x == 0) init_barriers(c, 8);
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < t; ++s) {
+      prefetch_tmap(&p.ta[s]);
+      prefetch_tmap(&p.tb[s]);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
+  const uint32_t tmem_base = *tmem_slot;
+
+  int last_phase[STAGES];
+  bool issued[STAGES];
+#pragma unroll
+  for (int s = 0; s < STAGES; ++s) { last_phase[s] = 0; issued[s] = false; }
+  bool mma_issued = false;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      Ring r;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+        int mt, nt;
+        raster_by_chunk(tile, p.tiles_m, p.tiles_n, p.axis, p.chunk_tiles, mt, nt);
+        const int m0 = mt * BM, n0 = nt * BN;
+        const int ch = (p.axis == 0 ? m0 : n0) / p.chunk;
+        for (int j = 0; ok && j < t; ++j) {
+          const int s = (ch + 1 + j) % t;              // ring order of this chunk
+          ok = produce_unit(c, r, &p.ta[s], &p.tb[s], nullptr, m0, n0, p.num_kb, last_phase, issued);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      Ring r;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+        for (int j = 0; ok && j < t; ++j) {
+          ok = wait_or_abort(c, c.acce0 + 8 * acc, acc_phase ^ 1u, WAIT_MMA_ACC_EMPTY);
+          if (!ok) break;
+          tc_fence_after();
+          ok = mma_unit(c, r, tmem_base + static_cast<uint32_t>(acc * BN), p.num_kb, mma_issued);
+          if (!ok) break;
+          umma_commit(c.accf0 + 8 * acc);
+          if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+        }
+      }
+    }
+  } else {
+    // epilogue warps 2..9: TMEM lane quadrant = warp % 4; warps 2..5 take columns 0..127 of the
+    // tile and warps 6..9 columns 128..255. Each thread keeps its row's 128 running sums.
+    const int quad = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const uint32_t stg = staging0 + static_cast<uint32_t>(warp - 2) * STAGING_PER_WARP;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true;
+    float sum[4][32];
+    for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+      int mt, nt;
+      raster_by_chunk(tile, p.tiles_m, p.tiles_n, p.axis, p.chunk_tiles, mt, nt);
+      const int m0 = mt * BM, n0 = nt * BN;
+      const int ch = (p.axis == 0 ? m0 : n0) / p.chunk;
+      for (int j = 0; j < t; ++j) {
+        ok = wait_or_abort(c, c.accf0 + 8 * acc, acc_phase, WAIT_EPI_ACC_FULL);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
+                               static_cast<uint32_t>(acc * BN + half * 128);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t v[32];
+          tmem_ld32(t_row + q * 32, v);
+          tmem_ld_wait();
+          if (j == 0) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) sum[q][i] = __uint_as_float(v[i]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) sum[q][i] = __fadd_rn(sum[q][i], __uint_as_float(v[i]));
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(c.acce0 + 8 * acc);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      }
+      if (!ok) break;
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        store_block32<OUT_BF16, AR>(p, stg, lane, sum[q], m0 + quad * 32, n0 + half * 128 + q * 32, ch);
+    }
+  }
+  teardown(c, warp, lane, last_phase, issued, mma_issued, tmem_base);
 }
 
 // ------------------------------------------------------------------ host side
@@ -331,21 +797,57 @@ bool encode_bf16_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t o
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Reserve the dynamic shared memory of a kernel once per device.
+template <typename K>
+tp_status reserve_smem(K kernel, size_t bytes, int* done_for) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return fail(TP_ECUDA, "cudaGetDevice failed");
+  if (dev >= 0 && dev < 64 && !done_for[dev]) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes)) != cudaSuccess)
+      return fail(TP_ECUDA, "cannot reserve %zu bytes of shared memory", bytes);
+    done_for[dev] = 1;
+  }
+  return TP_OK;
+}
+
 template <int EPI>
 tp_status launch(GemmParams& p, cudaStream_t s) {
   static int configured_for[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return fail(TP_ECUDA, "cudaGetDevice failed");
-  if (dev >= 0 && dev < 64 && !configured_for[dev]) {
-    if (cudaFuncSetAttribute(gemm_tcgen05_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(SMEM_BYTES)) != cudaSuccess)
-      return fail(TP_ECUDA, "cannot reserve %zu bytes of shared memory", SMEM_BYTES);
-    configured_for[dev] = 1;
-  }
+  if (tp_status st = reserve_smem(gemm_tcgen05_kernel<EPI>, GEMM_SMEM, configured_for)) return st;
   const int sms = sm_count();
   const int grid = p.num_tiles < sms ? p.num_tiles : sms;
-  gemm_tcgen05_kernel<EPI><<<grid, THREADS, SMEM_BYTES, s>>>(p);
+  gemm_tcgen05_kernel<EPI><<<grid, GEMM_THREADS, GEMM_SMEM, s>>>(p);
   return check_launch("gemm_tcgen05_kernel");
+}
+
+template <int EPI>
+tp_status launch_pair(GemmParams& p, cudaStream_t s) {
+  static int configured_for[64] = {};
+  if (tp_status st = reserve_smem(gemm_pair_kernel<EPI>, PAIR_SMEM, configured_for)) return st;
+  const int sms = sm_count();
+  const int tiles = p.groups * ((p.M + 2 * BM - 1) / (2 * BM)) * p.tiles_n;
+  int grid = 2 * tiles < sms ? 2 * tiles : (sms & ~1);
+  if (grid < 2) grid = 2;
+  gemm_pair_kernel<EPI><<<grid, GEMM_THREADS, PAIR_SMEM, s>>>(p);
+  return check_launch("gemm_pair_kernel");
+}
+
+template <bool OUT_BF16, bool AR>
+tp_status launch_ring(RingGemmParams& p, cudaStream_t s) {
+  static int configured_for[64] = {};
+  if (tp_status st = reserve_smem(gemm_ring_kernel<OUT_BF16, AR>, RING_SMEM, configured_for)) return st;
+  const int sms = sm_count();
+  const int grid = p.num_tiles < sms ? p.num_tiles : sms;
+  gemm_ring_kernel<OUT_BF16, AR><<<grid, RING_THREADS, RING_SMEM, s>>>(p);
+  return check_launch("gemm_ring_kernel");
+}
+
+tp_status check_operands(int n, const uint16_t* const* a, const uint16_t* const* b, void* const* c) {
+  for (int i = 0; i < n; ++i) {
+    if (a[i] == nullptr || b[i] == nullptr || c[i] == nullptr) return fail(TP_EINVAL, "null GEMM operand %d", i);
+    if (!aligned16(a[i]) || !aligned16(b[i]) || !aligned16(c[i])) return fail(TP_EALIGN, "GEMM operand %d not 16-byte aligned", i);
+  }
+  return TP_OK;
 }
 
 }  // namespace
@@ -357,10 +859,7 @@ tp_status grouped_gemm(const GemmArgs& g, cudaStream_t s) {
   const bool swiglu = g.epi == EPI_SWIGLU;
   if (g.K % 8 || g.N % 8 || g.lda % 8 || g.ldb % 8) return fail(TP_EALIGN, "K, N and row strides must be multiples of 8");
   if (g.lda < g.K || g.ldb < (swiglu ? 2 * g.N : g.N)) return fail(TP_ESHAPE, "row stride shorter than the row");
-  for (int i = 0; i < g.groups; ++i) {
-    if (g.a[i] == nullptr || g.b[i] == nullptr || g.c[i] == nullptr) return fail(TP_EINVAL, "null GEMM operand %d", i);
-    if (!aligned16(g.a[i]) || !aligned16(g.b[i]) || !aligned16(g.c[i])) return fail(TP_EALIGN, "GEMM operand %d not 16-byte aligned", i);
-  }
+  if (tp_status st = check_operands(g.groups, g.a, g.b, g.c)) return st;
   GemmParams p;
   std::memset(&p, 0, sizeof(p));
   const int tile_n = swiglu ? BN / 2 : BN;
@@ -387,6 +886,16 @@ tp_status grouped_gemm(const GemmArgs& g, cudaStream_t s) {
   p.status = status_word();
   p.budget = wait_budget();
   if (p.status == nullptr) return fail(TP_ECUDA, "cannot resolve the device status word");
+  // CTA pairs for problems with at least one full 256-row tile per group.
+  if (g.M >= 2 * BM) {
+    switch (g.epi) {
+      case EPI_F32: return launch_pair<EPI_F32>(p, s);
+      case EPI_BF16: return launch_pair<EPI_BF16>(p, s);
+      case EPI_GELU: return launch_pair<EPI_GELU>(p, s);
+      case EPI_GELU_TANH: return launch_pair<EPI_GELU_TANH>(p, s);
+      case EPI_SWIGLU: return launch_pair<EPI_SWIGLU>(p, s);
+    }
+  }
   switch (g.epi) {
     case EPI_F32: return launch<EPI_F32>(p, s);
     case EPI_BF16: return launch<EPI_BF16>(p, s);
@@ -395,6 +904,53 @@ tp_status grouped_gemm(const GemmArgs& g, cudaStream_t s) {
     case EPI_SWIGLU: return launch<EPI_SWIGLU>(p, s);
   }
   return fail(TP_EINVAL, "bad epilogue");
+}
+
+bool ring_gemm_fits(int64_t M, int64_t N, int t, int axis) {
+  if (axis == 0) return M % t == 0 && (M / t) % BM == 0;
+  return N % t == 0 && (N / t) % BN == 0;
+}
+
+tp_status ring_gemm(const RingGemmArgs& g, cudaStream_t s) {
+  if (!valid_t(g.t)) return fail(TP_EINVAL, "t=%d outside 1..%d", g.t, TP_MAX_SHARDS);
+  if (g.M <= 0 || g.N <= 0 || g.K <= 0) return fail(TP_EINVAL, "non-positive GEMM size");
+  if (g.M > INT32_MAX / 2 || g.N > INT32_MAX / 2 || g.K > INT32_MAX / 2) return fail(TP_ESHAPE, "GEMM size too large");
+  if (g.op != RING_RS && g.op != RING_AR) return fail(TP_EINVAL, "fused GEMM reduces by RS or AR only");
+  const int axis = g.op == RING_AR ? 0 : g.axis;
+  if (!ring_gemm_fits(g.M, g.N, g.t, axis)) return fail(TP_EUNSUPPORTED, "chunks do not align with 128 x 256 tiles");
+  if (g.K % 8 || g.N % 8 || g.lda % 8 || g.ldb % 8) return fail(TP_EALIGN, "K, N and row strides must be multiples of 8");
+  if (g.lda < g.K || g.ldb < g.N) return fail(TP_ESHAPE, "row stride shorter than the row");
+  if (tp_status st = check_operands(g.t, g.a, g.b, g.out)) return st;
+  if ((g.resid && !aligned16(g.resid)) || (g.copy_bf16 && !aligned16(g.copy_bf16)))
+    return fail(TP_EALIGN, "residual or bf16 copy not 16-byte aligned");
+  RingGemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  for (int i = 0; i < g.t; ++i) {
+    if (!encode_bf16_2d(&p.ta[i], g.a[i], g.K, g.M, g.lda, BK, BM))
+      return fail(TP_ECUDA, "cannot encode the TMA descriptor of A[%d]", i);
+    if (!encode_bf16_2d(&p.tb[i], g.b[i], g.N, g.K, g.ldb, 64, BK))
+      return fail(TP_ECUDA, "cannot encode the TMA descriptor of B[%d]", i);
+    p.out[i] = g.out[i];
+  }
+  p.resid = g.op == RING_AR ? g.resid : nullptr;
+  p.resid_bf16 = g.resid_dtype == TP_BF16;
+  p.copy_bf16 = g.op == RING_AR ? g.copy_bf16 : nullptr;
+  p.M = static_cast<int>(g.M);
+  p.N = static_cast<int>(g.N);
+  p.t = g.t;
+  p.axis = axis;
+  p.chunk = static_cast<int>(axis == 0 ? g.M / g.t : g.N / g.t);
+  p.chunk_tiles = axis == 0 ? p.chunk / BM : p.chunk / BN;
+  p.tiles_m = static_cast<int>(g.M / BM);
+  p.tiles_n = static_cast<int>((g.N + BN - 1) / BN);
+  p.num_tiles = p.tiles_m * p.tiles_n;
+  p.num_kb = static_cast<int>((g.K + BK - 1) / BK);
+  p.status = status_word();
+  p.budget = wait_budget();
+  if (p.status == nullptr) return fail(TP_ECUDA, "cannot resolve the device status word");
+  const bool bf16 = g.out_dtype == TP_BF16;
+  if (g.op == RING_AR) return bf16 ? launch_ring<true, true>(p, s) : launch_ring<false, true>(p, s);
+  return bf16 ? launch_ring<true, false>(p, s) : launch_ring<false, false>(p, s);
 }
 
 }  // namespace tpx
