@@ -323,22 +323,50 @@ def run_gpu(args) -> int:
     del partials, rs_out
 
     # ---- end to end through tp_mlp_fwd with host buffers --------------------------------------
+    # Every step copies its input X from pinned host memory and reads its result back (one replica
+    # of the reduced output). As a serving loop would, the copies run on their own streams and overlap
+    # the neighbouring steps' compute: copy-in of step i+1 || tp_mlp_fwd of step i || copy-out of step
+    # i-1, with two buffer sets and events guarding every reuse.
     x_host = X.cpu().pin_memory()
-    y_host = torch.empty((N_TOK, H), dtype=torch.float32).pin_memory()
-    x_dev = torch.empty_like(X)
-    for _ in range(max(1, min(args.warmup, 3))):
-        x_dev.copy_(x_host, non_blocking=True)
-        tp.tp_mlp_fwd(x_dev, N_TOK, H, F, T, tp.TP_ACT_SWIGLU, w_in, w_down, z, None, tp.TP_OUT_RS_AG, out)
-        y_host.copy_(out[0], non_blocking=True)
+    y_host = [torch.empty((N_TOK, H), dtype=torch.float32).pin_memory() for _ in range(2)]
+    x_dev = [torch.empty_like(X) for _ in range(2)]
+    outs = [out, [torch.empty((N_TOK, H), device=dev) for _ in range(T)]]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    for e in ev_comp + ev_out:
+        e.record(stream)
+
+    def e2e_steps(n):
+        for i in range(n):
+            b = i & 1
+            with torch.cuda.stream(s_in):
+                s_in.wait_event(ev_comp[b])                  # step i-2 no longer reads x_dev[b]
+                x_dev[b].copy_(x_host, non_blocking=True)
+                ev_in[b].record(s_in)
+            stream.wait_event(ev_in[b])
+            stream.wait_event(ev_out[b])                     # step i-2's result has been read back
+            tp.tp_mlp_fwd(x_dev[b], N_TOK, H, F, T, tp.TP_ACT_SWIGLU, w_in, w_down, z, None, tp.TP_OUT_RS_AG,
+                          outs[b], stream)
+            ev_comp[b].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_comp[b])
+                y_host[b].copy_(outs[b][0], non_blocking=True)
+                ev_out[b].record(s_out)
+
+    e2e_steps(max(2, min(args.warmup, 4)))
+    torch.cuda.synchronize()
     e_start, e_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
-    e_start.record(stream)
-    for _ in range(args.steps):
-        x_dev.copy_(x_host, non_blocking=True)
-        tp.tp_mlp_fwd(x_dev, N_TOK, H, F, T, tp.TP_ACT_SWIGLU, w_in, w_down, z, None, tp.TP_OUT_RS_AG, out)
-        y_host.copy_(out[0], non_blocking=True)
+    e_start.record(s_in)
+    stream.wait_event(e_start)
+    s_out.wait_event(e_start)
+    e2e_steps(args.steps)
+    stream.wait_event(ev_out[0])
+    stream.wait_event(ev_out[1])
     e_stop.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e_start.elapsed_time(e_stop)
@@ -387,7 +415,9 @@ def run_gpu(args) -> int:
                              "reduce_scatter_gbs": rs_gbs},
             "roofline": roofline, "roofline_fused_row_reduce": fused_roof, "roofline_reduce_scatter": roofline_rs,
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": X.numel() * 2,
-                    "d2h_bytes_per_step": N_TOK * H * 4},
+                    "d2h_bytes_per_step": N_TOK * H * 4, "ms_per_step": e2e_ms / args.steps,
+                    "how": "tp_mlp_fwd per step; pinned H2D of X and D2H of one reduced replica on separate "
+                           "streams, double-buffered, overlapping the neighbouring steps"},
             "gpu_launches": 2 * args.steps,
             "clocks": clk,
         }
@@ -400,6 +430,134 @@ def run_gpu(args) -> int:
     return 0
 
 
+# ------------------------------------------------------------------------------ other workloads
+def _time_ms(fn, iters: int, warmup: int = 3) -> float:
+    """Average device time of fn() over `iters` back-to-back calls (CUDA events, current stream)."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(iters):
+        fn()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / iters
+
+
+def run_sweep(args) -> int:
+    """The collective sweep: ReduceScatter, AllGather and AllReduce in ring order over t in {2,4,8} shard
+    buffers, fp32 and bf16, payload M = 1 MiB .. 1 GiB in powers of 4 (M = each shard's full buffer for
+    RS/AR, the gathered tensor for AG). GB/s = algorithmic bytes / time: RS and AG (t+1)M, AR 2tM."""
+    import torch
+    import tensor_sharded_matmul_b200 as tp
+    hbm_peak = _peaks()[0]
+    torch.cuda.set_device(0)
+    for t in (2, 4, 8):
+        for dt in ("f32", "bf16"):
+            es = 4 if dt == "f32" else 2
+            tdt = torch.float32 if dt == "f32" else torch.bfloat16
+            for mib in (1, 4, 16, 64, 256, 1024):
+                elems = mib * (1 << 20) // es
+                cols = 4096 if elems >= 4096 * 64 else 256
+                rows = elems // cols
+                for op in ("RS", "AG", "AR"):
+                    if op == "AG":
+                        ins = [torch.empty((rows // t, cols), dtype=tdt, device="cuda").normal_() for _ in range(t)]
+                        outs = [torch.empty((rows, cols), dtype=tdt, device="cuda") for _ in range(t)]
+                        fn = lambda: tp.tp_all_gather(ins, outs, rows, cols, 0, tp.TP_F32 if dt == "f32" else tp.TP_BF16, t)  # noqa: E731
+                        nbytes = (t + 1) * mib * (1 << 20)
+                    else:
+                        ins = [torch.empty((rows, cols), dtype=tdt, device="cuda").normal_() for _ in range(t)]
+                        shape = (rows // t, cols) if op == "RS" else (rows, cols)
+                        outs = [torch.empty(shape, dtype=tdt, device="cuda") for _ in range(t)]
+                        code = tp.TP_F32 if dt == "f32" else tp.TP_BF16
+                        if op == "RS":
+                            fn = lambda: tp.tp_reduce_scatter(ins, outs, rows, cols, 0, code, t)  # noqa: E731
+                            nbytes = (t + 1) * mib * (1 << 20)
+                        else:
+                            fn = lambda: tp.tp_all_reduce(ins, outs, rows, cols, code, t)  # noqa: E731
+                            nbytes = 2 * t * mib * (1 << 20)
+                    iters = max(5, min(200, int(2e9 / nbytes)))
+                    ms = _time_ms(fn, iters)
+                    gbs = nbytes / (ms * 1e-3) / 1e9
+                    bus = (t - 1) / t * mib * (1 << 20) * (2 if op == "AR" else 1) / (ms * 1e-3) / 1e9
+                    _emit({"config": "collective_sweep", "op": op, "t": t, "dtype": dt, "payload_mib": mib,
+                           "ms": ms, "gbs": gbs, "frac_hbm": gbs / hbm_peak, "ring_bus_gbs": bus})
+                    del ins, outs
+                    torch.cuda.empty_cache()
+    return 0
+
+
+def run_cases(args) -> int:
+    """The four sharded-matmul cases of C[B,F] = X[B,D] W[D,F] at B=D=8192, F=28672 over t=4 shards,
+    every strategy; TFLOP/s counts the FLOPs executed (case 2 AllGather computes C on every shard)."""
+    import torch
+    import synthetic as S
+    import tensor_sharded_matmul_b200 as tp
+    torch.cuda.set_device(0)
+    B, D, F, t = 8192, 8192, 28672, 4
+    X, W = S.case_operands(seed=0, device="cuda")
+    peak = _peaks()[1]
+    shard = {1: (list(X.chunk(t, 0)), [W] * t), 2: (list(X.chunk(t, 1)), [W] * t),
+             3: (list(X.chunk(t, 1)), list(W.chunk(t, 0))), 4: (list(X.chunk(t, 0)), list(W.chunk(t, 1)))}
+    names = {(1, 0): "local", (2, 0): "allgather", (2, 1): "allreduce", (3, 0): "allreduce", (3, 1): "rs_b",
+             (3, 2): "rs_f", (4, 0): "gather_x", (4, 1): "gather_w"}
+    shapes = {(1, 0): (B // t, F), (2, 0): (B, F), (2, 1): (B, F), (3, 0): (B, F), (3, 1): (B // t, F),
+              (3, 2): (B, F // t), (4, 0): (B, F // t), (4, 1): (B // t, F)}
+    for (case_id, strategy), name in names.items():
+        xs, ws = shard[case_id]
+        xs = [x.contiguous() for x in xs]
+        ws = [w.contiguous() for w in ws] if case_id in (3, 4) else ws
+        c = [torch.empty(shapes[(case_id, strategy)], device="cuda") for _ in range(t)]
+        nbytes = tp.tp_sharded_matmul_ws_bytes(case_id, strategy, B, D, F, t)
+        wsb = torch.empty(max(nbytes, 256), dtype=torch.uint8, device="cuda")
+        fn = lambda: tp.tp_sharded_matmul(case_id, strategy, xs, ws, B, D, F, t, c, tp.TP_F32, wsb, nbytes)  # noqa: E731
+        ms = _time_ms(fn, 10)
+        flops = 2.0 * B * D * F * (t if (case_id, strategy) == (2, 0) else 1)
+        _emit({"config": "sharded_matmul", "case": case_id, "strategy": name, "ms": ms,
+               "tflops_executed": flops / (ms * 1e-3) / 1e12, "frac_bf16_peak": flops / (ms * 1e-3) / 1e12 / peak})
+        del c, wsb, xs, ws
+        torch.cuda.empty_cache()
+    return 0
+
+
+def run_layer70b(args) -> int:
+    """One Llama-3-70B-shaped TP=8 layer on 2048 tokens without its attention core (QKV column GEMM,
+    W_O row GEMM + AllReduce + residual, SwiGLU MLP + AllReduce + residual)."""
+    import torch
+    import synthetic as S
+    import tensor_sharded_matmul_b200 as tp
+    torch.cuda.set_device(0)
+    N, h, n_h, n_kv, d_h, F, t = 2048, 8192, 64, 8, 128, 28672, 8
+    L = S.llama70b_layer(seed=0, device="cuda")
+    qkv_w = (n_h // t + 2 * (n_kv // t)) * d_h
+    w_qkv = torch.empty((t, h, qkv_w), dtype=torch.bfloat16, device="cuda")
+    w_o = torch.empty((t, n_h * d_h // t, h), dtype=torch.bfloat16, device="cuda")
+    w_gu = torch.empty((t, h, 2 * F // t), dtype=torch.bfloat16, device="cuda")
+    w_down = torch.empty((t, F // t, h), dtype=torch.bfloat16, device="cuda")
+    tp.tp_shard_qkv(L["Wq"], n_h * d_h, L["Wk"], n_kv * d_h, L["Wv"], n_kv * d_h, h, n_h, n_kv, d_h, t, w_qkv)
+    tp.tp_shard_rows(L["Wo"], h, n_h * d_h, h, t, w_o)
+    tp.tp_shard_gate_up(L["Wg"], F, L["Wu"], F, h, F, t, w_gu)
+    tp.tp_shard_rows(L["Wd"], h, F, h, t, w_down)
+    o = [L["O"][:, r * n_h * d_h // t:(r + 1) * n_h * d_h // t].contiguous() for r in range(t)]
+    X = L["X"]
+    del L
+    qkv = torch.empty((t, N, qkv_w), dtype=torch.bfloat16, device="cuda")
+    h1 = [torch.empty((N, h), device="cuda") for _ in range(t)]
+    h1b = torch.empty((N, h), dtype=torch.bfloat16, device="cuda")
+    z = torch.empty((t, N, F // t), dtype=torch.bfloat16, device="cuda")
+    y = [torch.empty((N, h), device="cuda") for _ in range(t)]
+    fn = lambda: tp.tp_layer_fwd(X, o, N, h, n_h, n_kv, d_h, F, t, w_qkv, w_o, w_gu, w_down, qkv, h1, h1b, z,  # noqa: E731
+                                 None, y)
+    ms = _time_ms(fn, 50)
+    flops = 2.0 * N * (h * qkv_w * t + n_h * d_h * h + h * 2 * F + F * h)
+    _emit({"config": "llama70b_tp8_layer", "tokens": N, "ms": ms, "gflop": flops / 1e9,
+           "tflops": flops / (ms * 1e-3) / 1e12, "frac_bf16_peak": flops / (ms * 1e-3) / 1e12 / _peaks()[1]})
+    return 0
+
+
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -407,11 +565,19 @@ def main(argv=None) -> int:
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (profiling runs)")
+    ap.add_argument("--config", choices=["mlp8b", "sweep", "cases", "layer70b"], default="mlp8b",
+                    help="mlp8b: the headline step (one JSON line); the others print one line per measurement")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
+    if args.config == "sweep":
+        return run_sweep(args)
+    if args.config == "cases":
+        return run_cases(args)
+    if args.config == "layer70b":
+        return run_layer70b(args)
     return run_gpu(args)
 
 

@@ -66,6 +66,7 @@ constexpr uint32_t PAIR_B_STAGE = 128 * BK * 2;  // 16 KiB: two 64-wide boxes
 constexpr size_t PAIR_SMEM = 1024 + PAIR_STAGES * (PAIR_A_STAGE + PAIR_B_STAGE) + 256;
 constexpr uint32_t IDESC_PAIR = idesc_bf16_f32(2 * BM, BN, /*a_mn=*/false, /*b_mn=*/true);
 constexpr size_t RING_SMEM = 1024 + STAGES * (A_STAGE + B_STAGE) + 8 * STAGING_PER_WARP + 256;
+constexpr size_t RING_PAIR_SMEM = 1024 + PAIR_STAGES * (PAIR_A_STAGE + PAIR_B_STAGE) + 8 * STAGING_PER_WARP + 256;
 
 // ------------------------------------------------------------------ shared pipeline pieces
 struct Ring {
@@ -83,6 +84,7 @@ struct Ctl {
   volatile uint32_t* abort_flag;
   uint32_t* status;
   unsigned long long budget;
+  uint64_t b_policy;                       // L2 policy of the B (weight) loads
 };
 
 __device__ __forceinline__ bool wait_or_abort(const Ctl& c, uint32_t bar, uint32_t parity, uint32_t site) {
@@ -94,7 +96,7 @@ __device__ __forceinline__ bool wait_or_abort(const Ctl& c, uint32_t bar, uint32
 
 // Lays out barriers and the TMEM slot after the operand stages (and the staging area, if any).
 __device__ __forceinline__ Ctl setup_ctl(uint8_t* smem, uint32_t extra_bytes, uint32_t*& tmem_slot, uint32_t* status,
-                                         unsigned long long budget) {
+                                         unsigned long long budget, bool keep_b) {
   Ctl c;
   c.sA = smem;
   c.sB = smem + STAGES * A_STAGE;
@@ -108,6 +110,7 @@ __device__ __forceinline__ Ctl setup_ctl(uint8_t* smem, uint32_t extra_bytes, ui
   c.abort_flag = tmem_slot + 1;
   c.status = status;
   c.budget = budget;
+  c.b_policy = keep_b ? l2_policy_evict_last() : l2_policy_evict_normal();
   return c;
 }
 
@@ -138,14 +141,15 @@ __device__ __forceinline__ bool produce_unit(const Ctl& c, Ring& r, const CUtens
     const uint32_t b_dst = smem_u32(c.sB + r.stage * B_STAGE);
     const int k0 = kb * BK;
     tma_load_2d(a_dst, a, k0, m0, fb);
+    // B (the weights) is re-read by every row-tile: keep its lines in L2 longest
     if (b2 != nullptr) {
-      tma_load_2d(b_dst + 0 * B_BOX, b, n0, k0, fb);
-      tma_load_2d(b_dst + 1 * B_BOX, b, n0 + 64, k0, fb);
-      tma_load_2d(b_dst + 2 * B_BOX, b2, n0, k0, fb);
-      tma_load_2d(b_dst + 3 * B_BOX, b2, n0 + 64, k0, fb);
+      tma_load_2d_hint(b_dst + 0 * B_BOX, b, n0, k0, fb, c.b_policy);
+      tma_load_2d_hint(b_dst + 1 * B_BOX, b, n0 + 64, k0, fb, c.b_policy);
+      tma_load_2d_hint(b_dst + 2 * B_BOX, b2, n0, k0, fb, c.b_policy);
+      tma_load_2d_hint(b_dst + 3 * B_BOX, b2, n0 + 64, k0, fb, c.b_policy);
     } else {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) tma_load_2d(b_dst + j * B_BOX, b, n0 + 64 * j, k0, fb);
+      for (int j = 0; j < 4; ++j) tma_load_2d_hint(b_dst + j * B_BOX, b, n0 + 64 * j, k0, fb, c.b_policy);
     }
     issued[r.stage] = true;
     last_phase[r.stage] = static_cast<int>(r.phase);
@@ -291,7 +295,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tcgen05_kernel(const __g
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint32_t* tmem_slot;
-  const Ctl c = setup_ctl(smem, 0, tmem_slot, p.status, p.budget);
+  const Ctl c = setup_ctl(smem, 0, tmem_slot, p.status, p.budget, false);
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
 
@@ -378,12 +382,170 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tcgen05_kernel(const __g
   teardown(c, warp, lane, last_phase, issued, mma_issued, tmem_base);
 }
 
+// ------------------------------------------------------------------ CTA-pair pipeline
+// The two CTAs of a cluster share 256-row tiles. Each CTA loads its 128 rows of A and its half of
+// B's 256 columns (SwiGLU: CTA 0 the gate half, CTA 1 the up half) into its own shared memory, and
+// the copies of both CTAs count on the leader's (CTA 0's) full barrier. The leader's single MMA
+// thread issues tcgen05.mma.cta_group::2 (M=256, N=256). Its commits arrive on the barrier at the
+// same offset in both CTAs (stage free, accumulator ready). Each CTA's TMEM receives its own 128
+// rows. The epilogue warps of BOTH CTAs release an accumulator on the leader's barrier.
+struct PairCtl {
+  uint8_t* sA;
+  uint8_t* sB;
+  uint32_t full0, empty0, accf0, acce0, drain;
+  uint32_t full0_leader, acce0_leader;       // shared::cluster addresses in CTA 0
+  volatile uint32_t* abort_flag;
+  uint32_t* status;
+  unsigned long long budget;
+  uint32_t rank;
+  uint64_t b_policy;                         // L2 policy of the B (weight) loads
+};
+
+struct PairRing {
+  int stage = 0;
+  uint32_t phase = 0;
+  __device__ __forceinline__ void advance() {
+    if (++stage == PAIR_STAGES) { stage = 0; phase ^= 1u; }
+  }
+};
+
+__device__ __forceinline__ PairCtl pair_setup(uint8_t* smem, uint32_t extra_bytes, uint32_t*& tmem_slot,
+                                              uint32_t epilogue_warps_per_cta, uint32_t* status,
+                                              unsigned long long budget, bool keep_b) {
+  PairCtl c;
+  c.sA = smem;
+  c.sB = smem + PAIR_STAGES * PAIR_A_STAGE;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(c.sB + PAIR_STAGES * PAIR_B_STAGE + extra_bytes);
+  c.full0 = smem_u32(bars);
+  c.empty0 = c.full0 + 8 * PAIR_STAGES;
+  c.accf0 = c.empty0 + 8 * PAIR_STAGES;
+  c.acce0 = c.accf0 + 16;
+  c.drain = c.acce0 + 16;
+  tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * PAIR_STAGES + 5);
+  c.abort_flag = tmem_slot + 1;
+  c.status = status;
+  c.budget = budget;
+  c.rank = cluster_ctarank();
+  c.b_policy = keep_b ? l2_policy_evict_last() : l2_policy_evict_normal();
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < PAIR_STAGES; ++s) {
+      mbar_init(c.full0 + 8 * s, 1);
+      mbar_init(c.empty0 + 8 * s, 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(c.accf0 + 8 * a, 1);
+      mbar_init(c.acce0 + 8 * a, 2 * epilogue_warps_per_cta);   // epilogue warps of both CTAs
+    }
+    mbar_init(c.drain, 1);
+    *c.abort_flag = 0u;
+    fence_mbar_init();
+  }
+  if (threadIdx.x / 32 == 1) {
+    tmem_alloc_pair(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();   // barriers of both CTAs initialised, TMEM allocated in both
+  tc_fence_after();
+  c.full0_leader = mapa_shared(c.full0, 0);
+  c.acce0_leader = mapa_shared(c.acce0, 0);
+  return c;
+}
+
+__device__ __forceinline__ bool pair_fail(const PairCtl& c, uint32_t site) {
+  if (!*c.abort_flag) record_timeout(c.status, site);
+  *c.abort_flag = 1u;
+  return false;
+}
+
+// Producer of one CTA: the num_kb k-blocks of one unit. m0 is this CTA's first row, nb its first
+// B column (two 64-wide boxes of `tb`).
+__device__ __forceinline__ bool pair_produce_unit(const PairCtl& c, PairRing& r, const CUtensorMap* ta, int m0,
+                                                  const CUtensorMap* tb, int nb, int num_kb) {
+  for (int kb = 0; kb < num_kb; ++kb) {
+    if (!mbar_wait_bounded(c.empty0 + 8 * r.stage, r.phase ^ 1u, c.budget, c.abort_flag))
+      return pair_fail(c, WAIT_PRODUCER_EMPTY);
+    if (c.rank == 0) mbar_arrive_expect_tx(c.full0 + 8 * r.stage, 2 * (PAIR_A_STAGE + PAIR_B_STAGE));
+    const uint32_t fb = c.full0_leader + 8 * r.stage;
+    const uint32_t a_dst = smem_u32(c.sA + r.stage * PAIR_A_STAGE);
+    const uint32_t b_dst = smem_u32(c.sB + r.stage * PAIR_B_STAGE);
+    const int k0 = kb * BK;
+    tma_load_2d_pair(a_dst, ta, k0, m0, fb);
+    tma_load_2d_pair_hint(b_dst, tb, nb, k0, fb, c.b_policy);
+    tma_load_2d_pair_hint(b_dst + B_BOX, tb, nb + 64, k0, fb, c.b_policy);
+    r.advance();
+  }
+  return true;
+}
+
+// Leader's MMA thread: wait until both CTAs' epilogues released accumulator `acc`.
+__device__ __forceinline__ bool pair_wait_acc_empty(const PairCtl& c, int acc, uint32_t parity) {
+  bool got = mbar_try_wait_cluster(c.acce0 + 8 * acc, parity);
+  if (!got) {
+    const long long t0 = clock64();
+    while (!(got = mbar_try_wait_cluster(c.acce0 + 8 * acc, parity))) {
+      if (*c.abort_flag || static_cast<unsigned long long>(clock64() - t0) > c.budget) break;
+    }
+  }
+  if (!got) return pair_fail(c, WAIT_MMA_ACC_EMPTY);
+  tc_fence_after();
+  return true;
+}
+
+// Leader's MMA thread: one unit's num_kb k-blocks into d_tmem (M=256 over the pair, N=256).
+__device__ __forceinline__ bool pair_mma_unit(const PairCtl& c, PairRing& r, uint32_t d_tmem, int num_kb,
+                                              bool& mma_issued) {
+  for (int kb = 0; kb < num_kb; ++kb) {
+    if (!mbar_wait_bounded(c.full0 + 8 * r.stage, r.phase, c.budget, c.abort_flag)) return pair_fail(c, WAIT_MMA_FULL);
+    tc_fence_after();
+    const uint32_t a_base = smem_u32(c.sA + r.stage * PAIR_A_STAGE);
+    const uint32_t b_base = smem_u32(c.sB + r.stage * PAIR_B_STAGE);
+#pragma unroll
+    for (int k = 0; k < BK / 16; ++k) {
+      const uint64_t ad = smem_desc_sw128(a_base + 32u * k, 16u, 1024u);
+      const uint64_t bd = smem_desc_sw128(b_base + 2048u * k, B_BOX, 1024u);
+      umma_bf16_pair(d_tmem, ad, bd, IDESC_PAIR, (kb | k) != 0 ? 1u : 0u);
+    }
+    mma_issued = true;
+    umma_commit_pair_mc(c.empty0 + 8 * r.stage, 0x3);   // frees the stage in both CTAs
+    r.advance();
+  }
+  return true;
+}
+
+// Epilogue warp: wait for accumulator `acc` in this CTA.
+__device__ __forceinline__ bool pair_wait_acc_full(const PairCtl& c, int acc, uint32_t parity) {
+  if (!mbar_wait_bounded(c.accf0 + 8 * acc, parity, c.budget, c.abort_flag)) return pair_fail(c, WAIT_EPI_ACC_FULL);
+  tc_fence_after();
+  return true;
+}
+
+// Epilogue warp: hand accumulator `acc` back to the leader's MMA thread.
+__device__ __forceinline__ void pair_release_acc(const PairCtl& c, int acc, int lane) {
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive_cluster(c.acce0_leader + 8 * acc);
+}
+
+// All pair MMAs complete (they read both CTAs' shared memory and write both TMEMs), then both
+// CTAs meet before either releases TMEM or exits.
+__device__ __forceinline__ void pair_teardown(const PairCtl& c, int warp, int lane, bool mma_issued,
+                                              uint32_t tmem_base) {
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1 && lane == 0 && c.rank == 0 && mma_issued) {
+    umma_commit_pair(c.drain);
+    if (!mbar_wait_bounded(c.drain, 0, 4000000000ull, nullptr)) record_timeout(c.status, WAIT_TEARDOWN);
+  }
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_pair(tmem_base, TMEM_COLS);
+}
+
 // ------------------------------------------------------------------ CTA-pair grouped GEMM
-// Same computation as gemm_tcgen05_kernel, on 256-row tiles shared by the two CTAs of a cluster.
-// Each CTA loads its 128 rows of A and its half of B's 256 columns (SwiGLU: CTA 0 the gate half, CTA 1
-// the up half) into its own shared memory. The copies of both CTAs count on the leader's barrier.
-// The leader's single MMA thread issues tcgen05.mma.cta_group::2 (M=256, N=256). Each CTA's TMEM
-// receives its own 128 rows, and each CTA's epilogue stores them.
+// Same computation as gemm_tcgen05_kernel on 256-row tiles shared by the two CTAs of a cluster.
 template <int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     gemm_pair_kernel(const __grid_constant__ GemmParams p) {
@@ -393,136 +555,48 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sA = smem;
-  uint8_t* sB = smem + PAIR_STAGES * PAIR_A_STAGE;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + PAIR_STAGES * PAIR_B_STAGE);
-  const uint32_t full0 = smem_u32(bars);
-  const uint32_t empty0 = full0 + 8 * PAIR_STAGES;
-  const uint32_t accf0 = empty0 + 8 * PAIR_STAGES;
-  const uint32_t acce0 = accf0 + 16;
-  const uint32_t drain = acce0 + 16;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * PAIR_STAGES + 5);
-  volatile uint32_t* abort_flag = tmem_slot + 1;
-
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  const uint32_t rank = cluster_ctarank();
-  const bool leader = rank == 0;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < PAIR_STAGES; ++s) {
-      mbar_init(full0 + 8 * s, 1);
-      mbar_init(empty0 + 8 * s, 1);
-    }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(accf0 + 8 * a, 1);
-      mbar_init(acce0 + 8 * a, 8);   // 4 epilogue warps in each CTA of the pair
-    }
-    mbar_init(drain, 1);
-    *abort_flag = 0u;
-    fence_mbar_init();
-  }
   if (warp == 0 && lane == 0) {
     for (int g = 0; g < p.groups; ++g) {
       prefetch_tmap(&p.ta[g]);
-      prefetch_tmap(rank == 1 && SWIGLU ? &p.tb2[g] : &p.tb[g]);
+      prefetch_tmap(&p.tb[g]);
+      if (SWIGLU) prefetch_tmap(&p.tb2[g]);
     }
   }
-  if (warp == 1) {
-    tmem_alloc_pair(smem_u32(tmem_slot), TMEM_COLS);
-    tmem_relinquish_pair();
-  }
-  tc_fence_before();
-  cluster_sync();   // barriers of both CTAs initialised, TMEM allocated
-  tc_fence_after();
+  uint32_t* tmem_slot;
+  const PairCtl c = pair_setup(smem, 0, tmem_slot, 4, p.status, p.budget, false);
   const uint32_t tmem_base = *tmem_slot;
-  const uint32_t full0_leader = mapa_shared(full0, 0);
-  const uint32_t acce0_leader = mapa_shared(acce0, 0);
   const int pair = blockIdx.x >> 1;
   const int pairs = gridDim.x >> 1;
   const int tiles_m = (p.M + TILE_M - 1) / TILE_M;
   const int row_tiles = p.groups * tiles_m;
   const int num_tiles = row_tiles * p.tiles_n;
-  const unsigned long long budget = p.budget;
   bool mma_issued = false;
 
   if (warp == 0) {
     if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      bool ok = true;
-      for (int tile = pair; ok && tile < num_tiles; tile += pairs) {
+      PairRing r;
+      for (int tile = pair; tile < num_tiles; tile += pairs) {
         int rt, nt;
         raster(tile, row_tiles, p.tiles_n, rt, nt);
         const int g = rt / tiles_m;
-        const int m0 = (rt - g * tiles_m) * TILE_M + static_cast<int>(rank) * BM;
+        const int m0 = (rt - g * tiles_m) * TILE_M + static_cast<int>(c.rank) * BM;
         const int n0 = nt * TILE_N;
-        const CUtensorMap* tb = SWIGLU ? (rank == 0 ? &p.tb[g] : &p.tb2[g]) : &p.tb[g];
-        const int nb = SWIGLU ? n0 : n0 + static_cast<int>(rank) * 128;
-        for (int kb = 0; kb < p.num_kb; ++kb) {
-          if (!mbar_wait_bounded(empty0 + 8 * stage, phase ^ 1u, budget, abort_flag)) {
-            if (!*abort_flag) record_timeout(p.status, WAIT_PRODUCER_EMPTY);
-            *abort_flag = 1u;
-            ok = false;
-            break;
-          }
-          if (leader) mbar_arrive_expect_tx(full0 + 8 * stage, 2 * (PAIR_A_STAGE + PAIR_B_STAGE));
-          const uint32_t fb = full0_leader + 8 * stage;
-          const uint32_t a_dst = smem_u32(sA + stage * PAIR_A_STAGE);
-          const uint32_t b_dst = smem_u32(sB + stage * PAIR_B_STAGE);
-          const int k0 = kb * BK;
-          tma_load_2d_pair(a_dst, &p.ta[g], k0, m0, fb);
-          tma_load_2d_pair(b_dst, tb, nb, k0, fb);
-          tma_load_2d_pair(b_dst + B_BOX, tb, nb + 64, k0, fb);
-          if (++stage == PAIR_STAGES) { stage = 0; phase ^= 1u; }
-        }
+        const CUtensorMap* tb = SWIGLU ? (c.rank == 0 ? &p.tb[g] : &p.tb2[g]) : &p.tb[g];
+        const int nb = SWIGLU ? n0 : n0 + static_cast<int>(c.rank) * 128;
+        if (!pair_produce_unit(c, r, &p.ta[g], m0, tb, nb, p.num_kb)) break;
       }
     }
   } else if (warp == 1) {
-    if (lane == 0 && leader) {
-      int stage = 0;
-      uint32_t phase = 0;
+    if (lane == 0 && c.rank == 0) {
+      PairRing r;
       int acc = 0;
       uint32_t acc_phase = 0;
-      bool ok = true;
-      for (int tile = pair; ok && tile < num_tiles; tile += pairs) {
-        // the epilogues of BOTH CTAs release an accumulator on the leader's barrier
-        bool got = mbar_try_wait_cluster(acce0 + 8 * acc, acc_phase ^ 1u);
-        if (!got) {
-          const long long t0 = clock64();
-          while (!(got = mbar_try_wait_cluster(acce0 + 8 * acc, acc_phase ^ 1u))) {
-            if (*abort_flag || static_cast<unsigned long long>(clock64() - t0) > budget) break;
-          }
-        }
-        if (!got) {
-          if (!*abort_flag) record_timeout(p.status, WAIT_MMA_ACC_EMPTY);
-          *abort_flag = 1u;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
-        for (int kb = 0; kb < p.num_kb; ++kb) {
-          if (!mbar_wait_bounded(full0 + 8 * stage, phase, budget, abort_flag)) {
-            if (!*abort_flag) record_timeout(p.status, WAIT_MMA_FULL);
-            *abort_flag = 1u;
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t a_base = smem_u32(sA + stage * PAIR_A_STAGE);
-          const uint32_t b_base = smem_u32(sB + stage * PAIR_B_STAGE);
-#pragma unroll
-          for (int k = 0; k < BK / 16; ++k) {
-            const uint64_t ad = smem_desc_sw128(a_base + 32u * k, 16u, 1024u);
-            const uint64_t bd = smem_desc_sw128(b_base + 2048u * k, B_BOX, 1024u);
-            umma_bf16_pair(d_tmem, ad, bd, IDESC_PAIR, (kb | k) != 0 ? 1u : 0u);
-          }
-          mma_issued = true;
-          umma_commit_pair_mc(empty0 + 8 * stage, 0x3);   // frees the stage in both CTAs
-          if (++stage == PAIR_STAGES) { stage = 0; phase ^= 1u; }
-        }
-        if (!ok) break;
-        umma_commit_pair_mc(accf0 + 8 * acc, 0x3);          // both halves of the accumulator ready
+      for (int tile = pair; tile < num_tiles; tile += pairs) {
+        if (!pair_wait_acc_empty(c, acc, acc_phase ^ 1u)) break;
+        if (!pair_mma_unit(c, r, tmem_base + static_cast<uint32_t>(acc * BN), p.num_kb, mma_issued)) break;
+        umma_commit_pair_mc(c.accf0 + 8 * acc, 0x3);   // both halves of the accumulator ready
         if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
       }
     }
@@ -534,14 +608,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
       int rt, nt;
       raster(tile, row_tiles, p.tiles_n, rt, nt);
       const int g = rt / tiles_m;
-      const int m0 = (rt - g * tiles_m) * TILE_M + static_cast<int>(rank) * BM;
+      const int m0 = (rt - g * tiles_m) * TILE_M + static_cast<int>(c.rank) * BM;
       const int n0 = nt * TILE_N;
-      if (!mbar_wait_bounded(accf0 + 8 * acc, acc_phase, budget, abort_flag)) {
-        if (!*abort_flag) record_timeout(p.status, WAIT_EPI_ACC_FULL);
-        *abort_flag = 1u;
-        break;
-      }
-      tc_fence_after();
+      if (!pair_wait_acc_full(c, acc, acc_phase)) break;
       const int row = m0 + quad * 32 + lane;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * BN);
       void* cbase = p.c[g];
@@ -554,26 +623,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
         const int col0 = n0 + ch * 32;
         if (row < p.M && col0 < p.N) store_row_chunk<EPI>(cbase, p.N, row, col0, v, u);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(acce0_leader + 8 * acc);
+      pair_release_acc(c, acc, lane);
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
   }
-
-  // teardown: all pair MMAs complete (they read both CTAs' shared memory and write both TMEMs),
-  // then both CTAs meet before either releases TMEM or exits.
-  __syncwarp();
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1 && lane == 0 && leader && mma_issued) {
-    umma_commit_pair(drain);
-    if (!mbar_wait_bounded(drain, 0, 4000000000ull, nullptr)) record_timeout(p.status, WAIT_TEARDOWN);
-  }
-  tc_fence_before();
-  cluster_sync();
-  tc_fence_after();
-  if (warp == 1) tmem_dealloc_pair(tmem_base, TMEM_COLS);
+  pair_teardown(c, warp, lane, mma_issued, tmem_base);
 }
 
 // ------------------------------------------------------------------ fused row GEMM + ring reduction
@@ -636,20 +690,21 @@ __device__ __forceinline__ void store_block32(const RingGemmParams& p, uint32_t 
         }
         for (int s = 0; s < p.t; ++s) {
           if constexpr (OUT_BF16)
-            *reinterpret_cast<uint2*>(static_cast<uint16_t*>(p.out[s]) + e) = make_uint2(pack2(x.x, x.y), pack2(x.z, x.w));
+            st_cs_v2(static_cast<uint16_t*>(p.out[s]) + e, make_uint2(pack2(x.x, x.y), pack2(x.z, x.w)));
           else
-            *reinterpret_cast<float4*>(static_cast<float*>(p.out[s]) + e) = x;
+            st_cs_v4(static_cast<float*>(p.out[s]) + e, make_uint4(__float_as_uint(x.x), __float_as_uint(x.y),
+                                                                  __float_as_uint(x.z), __float_as_uint(x.w)));
         }
-        if (p.copy_bf16 != nullptr)
-          *reinterpret_cast<uint2*>(p.copy_bf16 + e) = make_uint2(pack2(x.x, x.y), pack2(x.z, x.w));
+        if (p.copy_bf16 != nullptr) st_cs_v2(p.copy_bf16 + e, make_uint2(pack2(x.x, x.y), pack2(x.z, x.w)));
       } else {
         // ReduceScatter: chunk c lands in shard c's output, at its place inside the chunk
         const int64_t o = p.axis == 0 ? static_cast<int64_t>(row - c * p.chunk) * p.N + col
                                       : static_cast<int64_t>(row) * p.chunk + (col - c * p.chunk);
         if constexpr (OUT_BF16)
-          *reinterpret_cast<uint2*>(static_cast<uint16_t*>(p.out[c]) + o) = make_uint2(pack2(x.x, x.y), pack2(x.z, x.w));
+          st_cs_v2(static_cast<uint16_t*>(p.out[c]) + o, make_uint2(pack2(x.x, x.y), pack2(x.z, x.w)));
         else
-          *reinterpret_cast<float4*>(static_cast<float*>(p.out[c]) + o) = x;
+          st_cs_v4(static_cast<float*>(p.out[c]) + o, make_uint4(__float_as_uint(x.x), __float_as_uint(x.y),
+                                                                __float_as_uint(x.z), __float_as_uint(x.w)));
       }
     }
   }
@@ -661,7 +716,8 @@ __global__ void __launch_bounds__(RING_THREADS, 1) gemm_ring_kernel(const __grid
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint32_t* tmem_slot;
-  const Ctl c = setup_ctl(smem, 8 * STAGING_PER_WARP, tmem_slot, p.status, p.budget);
+  // the fused kernel re-reads every shard's weight panels from each chunk: keep them in L2
+  const Ctl c = setup_ctl(smem, 8 * STAGING_PER_WARP, tmem_slot, p.status, p.budget, true);
   const uint32_t staging0 = smem_u32(smem + STAGES * (A_STAGE + B_STAGE));
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -770,6 +826,111 @@ __global__ void __launch_bounds__(RING_THREADS, 1) gemm_ring_kernel(const __grid
   teardown(c, warp, lane, last_phase, issued, mma_issued, tmem_base);
 }
 
+// Fused row GEMM + ring reduction on CTA pairs: the same ring-ordered epilogue as
+// gemm_ring_kernel, each CTA summing and storing its own 128 rows of a 256 x 256 pair tile.
+template <bool OUT_BF16, bool AR>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(RING_THREADS, 1)
+    gemm_ring_pair_kernel(const __grid_constant__ RingGemmParams p) {
+  constexpr int TILE_M = 2 * BM;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const int t = p.t;
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < t; ++s) {
+      prefetch_tmap(&p.ta[s]);
+      prefetch_tmap(&p.tb[s]);
+    }
+  }
+  uint32_t* tmem_slot;
+  // the fused kernel re-reads every shard's weight panels from each chunk: keep them in L2
+  const PairCtl c = pair_setup(smem, 8 * STAGING_PER_WARP, tmem_slot, 8, p.status, p.budget, true);
+  const uint32_t tmem_base = *tmem_slot;
+  const uint32_t staging0 = smem_u32(smem + PAIR_STAGES * (PAIR_A_STAGE + PAIR_B_STAGE));
+  const int pair = blockIdx.x >> 1;
+  const int pairs = gridDim.x >> 1;
+  const int tiles_m = (p.M + TILE_M - 1) / TILE_M;
+  const int num_tiles = tiles_m * p.tiles_n;
+  bool mma_issued = false;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      PairRing r;
+      bool ok = true;
+      for (int tile = pair; ok && tile < num_tiles; tile += pairs) {
+        int mt, nt;
+        raster_by_chunk(tile, tiles_m, p.tiles_n, p.axis, p.chunk_tiles, mt, nt);
+        const int ch = (p.axis == 0 ? mt * TILE_M : nt * BN) / p.chunk;
+        const int m0 = mt * TILE_M + static_cast<int>(c.rank) * BM;
+        const int nb = nt * BN + static_cast<int>(c.rank) * 128;
+        for (int j = 0; ok && j < t; ++j) {
+          const int s = (ch + 1 + j) % t;              // ring order of this chunk
+          ok = pair_produce_unit(c, r, &p.ta[s], m0, &p.tb[s], nb, p.num_kb);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && c.rank == 0) {
+      PairRing r;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = pair; ok && tile < num_tiles; tile += pairs) {
+        for (int j = 0; ok && j < t; ++j) {
+          ok = pair_wait_acc_empty(c, acc, acc_phase ^ 1u);
+          if (!ok) break;
+          ok = pair_mma_unit(c, r, tmem_base + static_cast<uint32_t>(acc * BN), p.num_kb, mma_issued);
+          if (!ok) break;
+          umma_commit_pair_mc(c.accf0 + 8 * acc, 0x3);
+          if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+        }
+      }
+    }
+  } else {
+    const int quad = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const uint32_t stg = staging0 + static_cast<uint32_t>(warp - 2) * STAGING_PER_WARP;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true;
+    float sum[4][32];
+    for (int tile = pair; ok && tile < num_tiles; tile += pairs) {
+      int mt, nt;
+      raster_by_chunk(tile, tiles_m, p.tiles_n, p.axis, p.chunk_tiles, mt, nt);
+      const int ch = (p.axis == 0 ? mt * TILE_M : nt * BN) / p.chunk;
+      const int m0 = mt * TILE_M + static_cast<int>(c.rank) * BM;
+      const int n0 = nt * BN;
+      for (int j = 0; j < t; ++j) {
+        ok = pair_wait_acc_full(c, acc, acc_phase);
+        if (!ok) break;
+        const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
+                               static_cast<uint32_t>(acc * BN + half * 128);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t v[32];
+          tmem_ld32(t_row + q * 32, v);
+          tmem_ld_wait();
+          if (j == 0) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) sum[q][i] = __uint_as_float(v[i]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) sum[q][i] = __fadd_rn(sum[q][i], __uint_as_float(v[i]));
+          }
+        }
+        pair_release_acc(c, acc, lane);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      }
+      if (!ok) break;
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        store_block32<OUT_BF16, AR>(p, stg, lane, sum[q], m0 + quad * 32, n0 + half * 128 + q * 32, ch);
+    }
+  }
+  pair_teardown(c, warp, lane, mma_issued, tmem_base);
+}
+
 // ------------------------------------------------------------------ host side
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -833,10 +994,19 @@ tp_status launch_pair(GemmParams& p, cudaStream_t s) {
 }
 
 template <bool OUT_BF16, bool AR>
-tp_status launch_ring(RingGemmParams& p, cudaStream_t s) {
+tp_status launch_ring(RingGemmParams& p, bool pair, cudaStream_t s) {
+  const int sms = sm_count();
+  if (pair) {
+    static int configured_for[64] = {};
+    if (tp_status st = reserve_smem(gemm_ring_pair_kernel<OUT_BF16, AR>, RING_PAIR_SMEM, configured_for)) return st;
+    const int tiles = ((p.M + 2 * BM - 1) / (2 * BM)) * p.tiles_n;
+    int grid = 2 * tiles < sms ? 2 * tiles : (sms & ~1);
+    if (grid < 2) grid = 2;
+    gemm_ring_pair_kernel<OUT_BF16, AR><<<grid, RING_THREADS, RING_PAIR_SMEM, s>>>(p);
+    return check_launch("gemm_ring_pair_kernel");
+  }
   static int configured_for[64] = {};
   if (tp_status st = reserve_smem(gemm_ring_kernel<OUT_BF16, AR>, RING_SMEM, configured_for)) return st;
-  const int sms = sm_count();
   const int grid = p.num_tiles < sms ? p.num_tiles : sms;
   gemm_ring_kernel<OUT_BF16, AR><<<grid, RING_THREADS, RING_SMEM, s>>>(p);
   return check_launch("gemm_ring_kernel");
@@ -940,7 +1110,9 @@ tp_status ring_gemm(const RingGemmArgs& g, cudaStream_t s) {
   p.t = g.t;
   p.axis = axis;
   p.chunk = static_cast<int>(axis == 0 ? g.M / g.t : g.N / g.t);
-  p.chunk_tiles = axis == 0 ? p.chunk / BM : p.chunk / BN;
+  // CTA pairs when every chunk is a whole number of 256-row (axis 0) or 256-column (axis 1) tiles
+  const bool pair = axis == 0 ? p.chunk % (2 * BM) == 0 : g.M >= 2 * BM;
+  p.chunk_tiles = axis == 0 ? p.chunk / (pair ? 2 * BM : BM) : p.chunk / BN;
   p.tiles_m = static_cast<int>(g.M / BM);
   p.tiles_n = static_cast<int>((g.N + BN - 1) / BN);
   p.num_tiles = p.tiles_m * p.tiles_n;
@@ -949,8 +1121,8 @@ tp_status ring_gemm(const RingGemmArgs& g, cudaStream_t s) {
   p.budget = wait_budget();
   if (p.status == nullptr) return fail(TP_ECUDA, "cannot resolve the device status word");
   const bool bf16 = g.out_dtype == TP_BF16;
-  if (g.op == RING_AR) return bf16 ? launch_ring<true, true>(p, s) : launch_ring<false, true>(p, s);
-  return bf16 ? launch_ring<true, false>(p, s) : launch_ring<false, false>(p, s);
+  if (g.op == RING_AR) return bf16 ? launch_ring<true, true>(p, pair, s) : launch_ring<false, true>(p, pair, s);
+  return bf16 ? launch_ring<true, false>(p, pair, s) : launch_ring<false, false>(p, pair, s);
 }
 
 }  // namespace tpx

@@ -42,6 +42,11 @@ CASES = [
     (2, 256, 400, 264, tp.TP_OUT_AR, 0),      # ragged K (k/t = 200) and an N tail (264)
     (3, 384, 768, 512, tp.TP_OUT_RS_AG, 0),   # t without a specialised ring kernel
     (8, 2048, 8192, 8192, tp.TP_OUT_AR, 0),   # the 70B W_O shape: 1024 of k per shard
+    # chunks of 256 rows: the CTA-pair variant of the fused kernel
+    (2, 512, 512, 512, tp.TP_OUT_RS, 0),
+    (4, 1024, 1024, 520, tp.TP_OUT_AR, 0),    # with an N tail
+    (3, 768, 768, 512, tp.TP_OUT_RS_AG, 0),
+    (2, 384, 512, 512, tp.TP_OUT_RS, 1),      # axis 1 on pairs with a 128-row M tail
 ]
 
 
@@ -78,10 +83,11 @@ def test_fused_equals_unfused_bitwise_and_oracle(t, N, k, n, mode, axis):
             assert_close(f64(fused[r])[rows], Y, GEMM_TOL, f"replica {r}")
 
 
-def test_fused_ring_order_matches_the_oracle_bitwise():
+@pytest.mark.parametrize("t,N", [(4, 512), (4, 1024)])      # 128-row chunks (single CTA), 256 (pairs)
+def test_fused_ring_order_matches_the_oracle_bitwise(t, N):
     # Feed the oracle the GPU's own fp32 partials (from the unfused GEMM): the ring sum must match bit for
     # bit, which shows that the fused epilogue adds the shards in the ring order the pages imply.
-    t, N, k, n = 4, 512, 1024, 512
+    k, n = 1024, 512
     x, w = _operands(t, N, k, n, seed=77)
     fused = [torch.empty((N // t, n), device="cuda") for _ in range(t)]
     tp.tp_row_linear_reduce(x, N, k, n, t, w, tp.TP_OUT_RS, 0, fused)
