@@ -141,6 +141,14 @@ tp_status tp_all_gather(const void* const* in, void* const* out, int64_t rows, i
 tp_status tp_all_reduce(const void* const* in, void* const* out, int64_t rows, int64_t cols,
                         tp_dtype dtype, int t, void* stream);
 
+/* AllToAll ([CH05] §5.3 AllToAll; [CH06] §6.4): every in[i] is a [rows, cols] buffer, split into t
+ * pieces along split_axis; out[j] receives piece j of every shard, concatenated along concat_axis in
+ * shard order. Output shape: [t*rows, cols/t] (split 1, concat 0: moves the sharding from rows to
+ * columns, A[I_X, J] -> A[I, J_X]); [rows/t, t*cols] (split 0, concat 1); [rows, cols] otherwise.
+ * A bit copy: reads t*M, writes t*M. Buffers must not overlap. */
+tp_status tp_all_to_all(const void* const* in, void* const* out, int64_t rows, int64_t cols, int split_axis,
+                        int concat_axis, tp_dtype dtype, int t, void* stream);
+
 /* ------------------------------------------------------------------------------------------------
  * GEMMs on the tensor cores (bf16 inputs, fp32 accumulation)
  * ------------------------------------------------------------------------------------------------ */
@@ -192,6 +200,25 @@ tp_status tp_row_linear_reduce(const uint16_t* x, int64_t N, int64_t k, int64_t 
 tp_status tp_mlp_fwd(const uint16_t* x, int64_t N, int64_t h, int64_t F, int t, tp_act act,
                      const uint16_t* w_in, const uint16_t* w_down, uint16_t* z_ws, float* const* partials,
                      tp_reduce mode, float* const* out, void* stream);
+
+/* ------------------------------------------------------------------------------------------------
+ * Tensor + sequence parallelism ([TPSP] §序列并行：把剩下的激活也切开). In the replicated region each
+ * shard holds only its own block of tokens, x[r] = rows [rN/t, (r+1)N/t) of X. The entry g is an
+ * AllGather along tokens and the exit g-bar a ReduceScatter along tokens. Same bytes as pure TP.
+ * ------------------------------------------------------------------------------------------------ */
+/* Column-parallel linear whose input is the AllGather of the t token shards x[r] (bf16 [N/t, k], host
+ * array of device pointers): y[r] = act(AllGather(x) . w[r]), stacked [t][N][n/t] bf16, with w as in
+ * tp_column_linear. The gathered X is never materialised: every 128-row tile of the GEMM's input is
+ * read from the shard that holds it. Needs (N/t) % 128 == 0 (TP_EUNSUPPORTED otherwise). */
+tp_status tp_column_linear_sp(const uint16_t* const* x, int64_t N, int64_t k, int64_t n, int t, tp_act act,
+                              const uint16_t* w, uint16_t* y, void* stream);
+/* The MLP under TP+SP: out[r] (fp32 [N/t, h]) = rows r of act(AllGather(x) W_in) W_down, i.e.
+ * tp_column_linear_sp, then the row GEMM fused with the ReduceScatter along tokens. x[r] bf16 [N/t, h];
+ * w_in, w_down and z_ws as in tp_mlp_fwd. Bit-identical to tp_mlp_fwd(TP_OUT_RS) on the gathered X.
+ * Needs (N/t) % 128 == 0. */
+tp_status tp_mlp_fwd_sp(const uint16_t* const* x, int64_t N, int64_t h, int64_t F, int t, tp_act act,
+                        const uint16_t* w_in, const uint16_t* w_down, uint16_t* z_ws, float* const* out,
+                        void* stream);
 
 /* ------------------------------------------------------------------------------------------------
  * The four sharded-matmul cases of C[B,F] = X[B,D] . W[D,F] over t shards ([CH06] §6.2, §6.9

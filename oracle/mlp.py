@@ -96,3 +96,14 @@ def row_first_mlp(X, A_row_shards, act: str):
     t = len(A_row_shards)
     Xs = np.split(np.asarray(X, dtype=np.float64), t, axis=1)
     return sum(activate(matmul(x, a), act) for x, a in zip(Xs, A_row_shards))
+
+
+def sp_mlp(x_shards, W_in_shards, W_out_shards, act: str, device_model: bool = False):
+    """The MLP under tensor + sequence parallelism ("张量并行与序列并行", §序列并行：把剩下的激活也切开): each
+    shard holds its own block of tokens; the entry g gathers them along s (AllGather), the column and
+    row layers run as in pure TP, and the exit g-bar sums and re-splits along s (ReduceScatter).
+    Returns each shard's block of the output rows (fp64)."""
+    from .collectives import all_gather, reduce_scatter_f64
+    X = all_gather([np.asarray(x, dtype=np.float64) for x in x_shards], axis=0)[0]
+    U = mlp_partials(X, W_in_shards, W_out_shards, act, device_model)
+    return reduce_scatter_f64(U, axis=0)

@@ -36,6 +36,7 @@ EXPORTED = (
     "tp_num_sms", "tp_shard_cols", "tp_shard_rows", "tp_shard_gate_up", "tp_shard_qkv", "tp_reduce_scatter",
     "tp_all_gather", "tp_all_reduce", "tp_grouped_gemm", "tp_column_linear", "tp_row_linear", "tp_row_linear_reduce", "tp_mlp_fwd",
     "tp_sharded_matmul_ws_bytes", "tp_sharded_matmul", "tp_layer_fwd", "tp_mlp_fwd_noalloc",
+    "tp_column_linear_sp", "tp_mlp_fwd_sp", "tp_all_to_all",
 )
 
 _vp, _i64, _i32, _u64, _sz = C.c_void_p, C.c_int64, C.c_int, C.c_uint64, C.c_size_t
@@ -55,12 +56,15 @@ _SIGS = {
     "tp_reduce_scatter": (_i32, [_pp, _pp, _i64, _i64, _i32, _i32, _i32, _vp]),
     "tp_all_gather": (_i32, [_pp, _pp, _i64, _i64, _i32, _i32, _i32, _vp]),
     "tp_all_reduce": (_i32, [_pp, _pp, _i64, _i64, _i32, _i32, _vp]),
+    "tp_all_to_all": (_i32, [_pp, _pp, _i64, _i64, _i32, _i32, _i32, _i32, _vp]),
     "tp_grouped_gemm": (_i32, [_i32, _pp, _pp, _pp, _i64, _i64, _i64, _i32, _i32, _vp]),
     "tp_column_linear": (_i32, [_vp, _i64, _i64, _i64, _i32, _i32, _vp, _vp, _vp]),
     "tp_row_linear": (_i32, [_vp, _i64, _i64, _i64, _i32, _vp, _pp, _vp]),
     "tp_row_linear_reduce": (_i32, [_vp, _i64, _i64, _i64, _i32, _vp, _i32, _i32, _pp, _pp, _vp]),
     "tp_mlp_fwd": (_i32, [_vp, _i64, _i64, _i64, _i32, _i32, _vp, _vp, _vp, _pp, _i32, _pp, _vp]),
     "tp_mlp_fwd_noalloc": (_i32, [_vp, _i64, _i64, _i64, _i32, _i32, _vp, _vp, _i32, _pp, _vp]),
+    "tp_column_linear_sp": (_i32, [_pp, _i64, _i64, _i64, _i32, _i32, _vp, _vp, _vp]),
+    "tp_mlp_fwd_sp": (_i32, [_pp, _i64, _i64, _i64, _i32, _i32, _vp, _vp, _vp, _pp, _vp]),
     "tp_sharded_matmul_ws_bytes": (_sz, [_i32, _i32, _i64, _i64, _i64, _i32]),
     "tp_sharded_matmul": (_i32, [_i32, _i32, _pp, _pp, _i64, _i64, _i64, _i32, _pp, _i32, _vp, _sz, _vp]),
     "tp_layer_fwd": (_i32, [_vp, _pp, _i64, _i64, _i32, _i32, _i32, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _pp,
@@ -169,6 +173,10 @@ def tp_all_reduce(ins, outs, rows, cols, dtype, t, stream=None):
     _call("tp_all_reduce", _ptrs(ins), _ptrs(outs), rows, cols, dtype, t, _stream(stream))
 
 
+def tp_all_to_all(ins, outs, rows, cols, split_axis, concat_axis, dtype, t, stream=None):
+    _call("tp_all_to_all", _ptrs(ins), _ptrs(outs), rows, cols, split_axis, concat_axis, dtype, t, _stream(stream))
+
+
 # ---- GEMMs, MLP, cases, layer -----------------------------------------------------------------
 def tp_grouped_gemm(groups, a, b, c, M, N, K, act, c_dtype, stream=None):
     _call("tp_grouped_gemm", groups, _ptrs(a), _ptrs(b), _ptrs(c), M, N, K, act, c_dtype, _stream(stream))
@@ -200,6 +208,15 @@ def tp_mlp_fwd_noalloc(x, N, h, F, t, act, w_in, w_down, mode, out, stream=None)
 
 
 TP_MLP_NOALLOC_SCRATCH_BYTES = 32 << 20
+
+
+def tp_column_linear_sp(x, N, k, n, t, act, w, y, stream=None):
+    _call("tp_column_linear_sp", _ptrs(x), N, k, n, t, act, _ptr(w), _ptr(y), _stream(stream))
+
+
+def tp_mlp_fwd_sp(x, N, h, F, t, act, w_in, w_down, z_ws, out, stream=None):
+    _call("tp_mlp_fwd_sp", _ptrs(x), N, h, F, t, act, _ptr(w_in), _ptr(w_down), _ptr(z_ws), _ptrs(out),
+          _stream(stream))
 
 
 def tp_sharded_matmul_ws_bytes(case_id, strategy, B, D, F, t) -> int:

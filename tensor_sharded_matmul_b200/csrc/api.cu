@@ -196,6 +196,41 @@ tp_status tp_mlp_fwd(const uint16_t* x, int64_t N, int64_t h, int64_t F, int t, 
   return reduce_partials(partials, N, h, t, mode, out, nullptr, TP_F32, nullptr, s);     // g: the collective
 }
 
+tp_status tp_column_linear_sp(const uint16_t* const* x, int64_t N, int64_t k, int64_t n, int t, tp_act act,
+                              const uint16_t* w, uint16_t* y, void* stream) {
+  if (!valid_t(t)) return fail(TP_EINVAL, "t=%d outside 1..%d", t, TP_MAX_SHARDS);
+  if (x == nullptr || w == nullptr || y == nullptr) return fail(TP_EINVAL, "null pointer");
+  if (!valid_act(act)) return fail(TP_EINVAL, "bad activation");
+  if (N <= 0 || k <= 0 || n <= 0) return fail(TP_EINVAL, "non-positive size");
+  if (n % t || N % t) return fail(TP_EDIVIS, "t=%d does not divide n or the token count", t);
+  if ((N / t) % 128) return fail(TP_EUNSUPPORTED, "token shards must be multiples of 128 rows");
+  const int64_t n_shard = n / t;
+  const int64_t wn = act == TP_ACT_SWIGLU ? 2 * n_shard : n_shard;
+  GemmArgs g = gemm_args(t, N, n_shard, k, k, wn, epi_for(act, TP_BF16));
+  g.a_slices = t;
+  g.slice_rows = N / t;
+  for (int r = 0; r < t; ++r) {
+    g.a_slice[r] = x[r];
+    g.b[r] = w + r * k * wn;
+    g.c[r] = y + r * N * n_shard;
+  }
+  return grouped_gemm(g, static_cast<cudaStream_t>(stream));
+}
+
+tp_status tp_mlp_fwd_sp(const uint16_t* const* x, int64_t N, int64_t h, int64_t F, int t, tp_act act,
+                        const uint16_t* w_in, const uint16_t* w_down, uint16_t* z_ws, float* const* out,
+                        void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (!valid_t(t)) return fail(TP_EINVAL, "t=%d outside 1..%d", t, TP_MAX_SHARDS);
+  if (x == nullptr || w_in == nullptr || w_down == nullptr || z_ws == nullptr || out == nullptr)
+    return fail(TP_EINVAL, "null pointer");
+  if (F % t) return fail(TP_EDIVIS, "t=%d does not divide F=%lld", t, (long long)F);
+  // g: AllGather along tokens, fused into the column GEMM's operand loads
+  if (tp_status st = tp_column_linear_sp(x, N, h, F, t, act, w_in, z_ws, stream)) return st;
+  // g-bar: the row GEMM fused with the ReduceScatter along tokens
+  return fused_row_reduce(z_ws, N, F / t, h, t, w_down, TP_OUT_RS, 0, out, nullptr, TP_F32, nullptr, s);
+}
+
 size_t tp_sharded_matmul_ws_bytes(int case_id, int strategy, int64_t B, int64_t D, int64_t F, int t) {
   if (t < 1 || B <= 0 || D <= 0 || F <= 0) return 0;
   const size_t T = static_cast<size_t>(t);

@@ -194,6 +194,40 @@ __global__ void __launch_bounds__(256) ring_gather_kernel(const __grid_constant_
   }
 }
 
+// AllToAll: out[j] = concatenation along concat_axis of piece j (split along split_axis) of every
+// shard's buffer. Each output element has exactly one source; UNIT bytes are moved per step.
+struct A2AParams {
+  const void* in[TP_MAX_SHARDS];
+  void* out[TP_MAX_SHARDS];
+  int64_t rows, cols;        // each shard's input shape
+  int64_t pr, pc;            // piece shape
+  int64_t orow, ocol;        // each shard's output shape
+  int t, split, concat;
+};
+
+template <int ES, int UNIT>
+__global__ void __launch_bounds__(256) all_to_all_kernel(const __grid_constant__ A2AParams p) {
+  constexpr int EPU = UNIT / ES;
+  const int64_t per_out = p.orow * p.ocol / EPU;
+  const int64_t units = per_out * p.t;
+  for (int64_t u = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; u < units;
+       u += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int j = static_cast<int>(u / per_out);
+    const int64_t e = (u - j * per_out) * EPU;
+    const int64_t r = e / p.ocol, col = e - r * p.ocol;
+    const int i = static_cast<int>(p.concat == 0 ? r / p.pr : col / p.pc);      // source shard
+    const int64_t lr = p.concat == 0 ? r - i * p.pr : r;
+    const int64_t lc = p.concat == 0 ? col : col - i * p.pc;
+    const int64_t sr = p.split == 0 ? j * p.pr + lr : lr;
+    const int64_t sc = p.split == 0 ? lc : j * p.pc + lc;
+    const char* src = static_cast<const char*>(p.in[i]) + (sr * p.cols + sc) * ES;
+    char* dst = static_cast<char*>(p.out[j]) + e * ES;
+    if constexpr (UNIT == 16) st_v4(dst, ld_nc_v4(src));
+    else if constexpr (ES == 4) *reinterpret_cast<uint32_t*>(dst) = *reinterpret_cast<const uint32_t*>(src);
+    else *reinterpret_cast<uint16_t*>(dst) = *reinterpret_cast<const uint16_t*>(src);
+  }
+}
+
 int grid_for(int64_t units) {
   const int sms = sm_count();
   const int64_t cap = static_cast<int64_t>(sms) * 8;   // 8 x 256 threads: a full SM
@@ -288,11 +322,57 @@ tp_status ring_collective(const RingArgs& a, cudaStream_t stream) {
   return check_launch("ring_reduce_kernel");
 }
 
+tp_status all_to_all(const void* const* in, void* const* out, int64_t rows, int64_t cols, int split, int concat,
+                     tp_dtype dtype, int t, cudaStream_t stream) {
+  if (in == nullptr || out == nullptr) return fail(TP_EINVAL, "null pointer array");
+  if (!valid_t(t)) return fail(TP_EINVAL, "t=%d outside 1..%d", t, TP_MAX_SHARDS);
+  if (rows <= 0 || cols <= 0) return fail(TP_EINVAL, "non-positive size");
+  if ((split != 0 && split != 1) || (concat != 0 && concat != 1)) return fail(TP_EINVAL, "axes must be 0 or 1");
+  if (dtype != TP_F32 && dtype != TP_BF16) return fail(TP_EINVAL, "bad dtype");
+  if (split == 0 ? rows % t : cols % t) return fail(TP_EDIVIS, "t=%d does not divide the split dimension", t);
+  A2AParams p;
+  std::memset(&p, 0, sizeof(p));
+  bool all16 = true;
+  for (int i = 0; i < t; ++i) {
+    if (in[i] == nullptr || out[i] == nullptr) return fail(TP_EINVAL, "null shard pointer %d", i);
+    for (int k = 0; k < t; ++k)
+      if (i != k && in[i] == out[k]) return fail(TP_EINVAL, "AllToAll cannot run in place");
+    p.in[i] = in[i];
+    p.out[i] = out[i];
+    all16 = all16 && aligned16(in[i]) && aligned16(out[i]);
+  }
+  p.rows = rows; p.cols = cols; p.t = t; p.split = split; p.concat = concat;
+  p.pr = split == 0 ? rows / t : rows;
+  p.pc = split == 1 ? cols / t : cols;
+  p.orow = concat == 0 ? t * p.pr : p.pr;
+  p.ocol = concat == 1 ? t * p.pc : p.pc;
+  const int es = dtype == TP_F32 ? 4 : 2;
+  const int epu = 16 / es;
+  // a vector never straddles a piece: the piece width, both row lengths and every column offset
+  // are multiples of the vector length
+  const bool vec = all16 && p.pc % epu == 0 && cols % epu == 0 && p.ocol % epu == 0;
+  const int64_t units = t * p.orow * p.ocol / (vec ? epu : 1);
+  const int blocks = grid_for(units);
+  if (es == 4) {
+    if (vec) all_to_all_kernel<4, 16><<<blocks, 256, 0, stream>>>(p);
+    else all_to_all_kernel<4, 4><<<blocks, 256, 0, stream>>>(p);
+  } else {
+    if (vec) all_to_all_kernel<2, 16><<<blocks, 256, 0, stream>>>(p);
+    else all_to_all_kernel<2, 2><<<blocks, 256, 0, stream>>>(p);
+  }
+  return check_launch("all_to_all_kernel");
+}
+
 }  // namespace tpx
 
 using namespace tpx;
 
 extern "C" {
+
+tp_status tp_all_to_all(const void* const* in, void* const* out, int64_t rows, int64_t cols, int split_axis,
+                        int concat_axis, tp_dtype dtype, int t, void* stream) {
+  return all_to_all(in, out, rows, cols, split_axis, concat_axis, dtype, t, static_cast<cudaStream_t>(stream));
+}
 
 tp_status tp_reduce_scatter(const void* const* in, void* const* out, int64_t rows, int64_t cols, int axis,
                             tp_dtype dtype, int t, void* stream) {

@@ -60,6 +60,11 @@ struct GemmArgs {
   void* c[TP_MAX_SHARDS];            // [M, N] row-major, row stride N
   int64_t M, N, K, lda, ldb;
   EpiKind epi;
+  // Optional: A given as a_slices row slices [slice_rows, K] shared by every group (a[] is then
+  // ignored); row m of A is row m % slice_rows of a_slice[m / slice_rows].
+  int a_slices;
+  int64_t slice_rows;
+  const uint16_t* a_slice[TP_MAX_SHARDS];
 };
 tp_status grouped_gemm(const GemmArgs& g, cudaStream_t s);
 

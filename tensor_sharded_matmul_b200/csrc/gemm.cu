@@ -255,9 +255,23 @@ struct GemmParams {
   void* c[TP_MAX_SHARDS];
   int M, N, K;                      // N = output columns
   int groups, tiles_m, tiles_n, row_tiles, num_tiles, num_kb;
+  // A given as row slices shared by all groups (the sequence-parallel entry: A = AllGather of t
+  // row shards): row m of A is row m % slice_rows of ta[m / slice_rows]. 0 = one A per group.
+  int a_slices, slice_rows;
   uint32_t* status;
   unsigned long long budget;
 };
+
+// Tensor map and local row of A for a tile starting at row m0 of group g.
+__device__ __forceinline__ const CUtensorMap* a_view(const GemmParams& p, int g, int m0, int& am0) {
+  if (p.a_slices) {
+    const int sl = m0 / p.slice_rows;
+    am0 = m0 - sl * p.slice_rows;
+    return &p.ta[sl];
+  }
+  am0 = m0;
+  return &p.ta[g];
+}
 
 // Store 32 consecutive output columns [col0, col0+32) of one row.
 template <int EPI>
@@ -302,10 +316,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tcgen05_kernel(const __g
   if (threadIdx.x == 0) init_barriers(c, 4);
   if (warp == 0 && lane == 0) {
     for (int g = 0; g < p.groups; ++g) {
-      prefetch_tmap(&p.ta[g]);
       prefetch_tmap(&p.tb[g]);
       if (SWIGLU) prefetch_tmap(&p.tb2[g]);
     }
+    for (int g = 0; g < (p.a_slices ? p.a_slices : p.groups); ++g) prefetch_tmap(&p.ta[g]);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
@@ -330,7 +344,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tcgen05_kernel(const __g
         raster(tile, p.row_tiles, p.tiles_n, rt, nt);
         const int g = rt / p.tiles_m;
         const int m0 = (rt - g * p.tiles_m) * BM;
-        if (!produce_unit(c, r, &p.ta[g], &p.tb[g], SWIGLU ? &p.tb2[g] : nullptr, m0, nt * TILE_N, p.num_kb,
+        int am0;
+        const CUtensorMap* ta = a_view(p, g, m0, am0);
+        if (!produce_unit(c, r, ta, &p.tb[g], SWIGLU ? &p.tb2[g] : nullptr, am0, nt * TILE_N, p.num_kb,
                           last_phase, issued))
           break;
       }
@@ -559,10 +575,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
   const int lane = threadIdx.x % 32;
   if (warp == 0 && lane == 0) {
     for (int g = 0; g < p.groups; ++g) {
-      prefetch_tmap(&p.ta[g]);
       prefetch_tmap(&p.tb[g]);
       if (SWIGLU) prefetch_tmap(&p.tb2[g]);
     }
+    for (int g = 0; g < (p.a_slices ? p.a_slices : p.groups); ++g) prefetch_tmap(&p.ta[g]);
   }
   uint32_t* tmem_slot;
   const PairCtl c = pair_setup(smem, 0, tmem_slot, 4, p.status, p.budget, false);
@@ -585,7 +601,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
         const int n0 = nt * TILE_N;
         const CUtensorMap* tb = SWIGLU ? (c.rank == 0 ? &p.tb[g] : &p.tb2[g]) : &p.tb[g];
         const int nb = SWIGLU ? n0 : n0 + static_cast<int>(c.rank) * 128;
-        if (!pair_produce_unit(c, r, &p.ta[g], m0, tb, nb, p.num_kb)) break;
+        int am0;
+        const CUtensorMap* ta = a_view(p, g, m0, am0);
+        if (!pair_produce_unit(c, r, ta, am0, tb, nb, p.num_kb)) break;
       }
     }
   } else if (warp == 1) {
@@ -1029,12 +1047,29 @@ tp_status grouped_gemm(const GemmArgs& g, cudaStream_t s) {
   const bool swiglu = g.epi == EPI_SWIGLU;
   if (g.K % 8 || g.N % 8 || g.lda % 8 || g.ldb % 8) return fail(TP_EALIGN, "K, N and row strides must be multiples of 8");
   if (g.lda < g.K || g.ldb < (swiglu ? 2 * g.N : g.N)) return fail(TP_ESHAPE, "row stride shorter than the row");
-  if (tp_status st = check_operands(g.groups, g.a, g.b, g.c)) return st;
+  for (int i = 0; i < g.groups; ++i) {
+    if ((!g.a_slices && g.a[i] == nullptr) || g.b[i] == nullptr || g.c[i] == nullptr) return fail(TP_EINVAL, "null GEMM operand %d", i);
+    if ((!g.a_slices && !aligned16(g.a[i])) || !aligned16(g.b[i]) || !aligned16(g.c[i]))
+      return fail(TP_EALIGN, "GEMM operand %d not 16-byte aligned", i);
+  }
   GemmParams p;
   std::memset(&p, 0, sizeof(p));
   const int tile_n = swiglu ? BN / 2 : BN;
+  const bool pair = g.M >= 2 * BM && (g.a_slices == 0 || g.slice_rows % (2 * BM) == 0);
+  if (g.a_slices) {
+    if (g.a_slices > TP_MAX_SHARDS || g.slice_rows <= 0 || g.slice_rows % BM != 0 || g.slice_rows * g.a_slices != g.M)
+      return fail(TP_ESHAPE, "A row slices must tile M in multiples of %d rows", BM);
+    for (int i = 0; i < g.a_slices; ++i) {
+      if (g.a_slice[i] == nullptr) return fail(TP_EINVAL, "null A slice %d", i);
+      if (!aligned16(g.a_slice[i])) return fail(TP_EALIGN, "A slice %d not 16-byte aligned", i);
+      if (!encode_bf16_2d(&p.ta[i], g.a_slice[i], g.K, g.slice_rows, g.lda, BK, BM))
+        return fail(TP_ECUDA, "cannot encode the TMA descriptor of A slice %d", i);
+    }
+    p.a_slices = g.a_slices;
+    p.slice_rows = static_cast<int>(g.slice_rows);
+  }
   for (int i = 0; i < g.groups; ++i) {
-    if (!encode_bf16_2d(&p.ta[i], g.a[i], g.K, g.M, g.lda, BK, BM))
+    if (!g.a_slices && !encode_bf16_2d(&p.ta[i], g.a[i], g.K, g.M, g.lda, BK, BM))
       return fail(TP_ECUDA, "cannot encode the TMA descriptor of A[%d]", i);
     if (!encode_bf16_2d(&p.tb[i], g.b[i], g.N, g.K, g.ldb, 64, BK))
       return fail(TP_ECUDA, "cannot encode the TMA descriptor of B[%d]", i);
@@ -1056,8 +1091,8 @@ tp_status grouped_gemm(const GemmArgs& g, cudaStream_t s) {
   p.status = status_word();
   p.budget = wait_budget();
   if (p.status == nullptr) return fail(TP_ECUDA, "cannot resolve the device status word");
-  // CTA pairs for problems with at least one full 256-row tile per group.
-  if (g.M >= 2 * BM) {
+  // CTA pairs for problems with at least one full 256-row tile per group (and slices of whole pair tiles).
+  if (pair) {
     switch (g.epi) {
       case EPI_F32: return launch_pair<EPI_F32>(p, s);
       case EPI_BF16: return launch_pair<EPI_BF16>(p, s);

@@ -182,3 +182,31 @@ def test_shard_qkv_bit_exact(h, n_h, n_kv, d_h, t):
     torch.cuda.synchronize()
     ref = OL.shard_qkv(S.bf16_bits(Wq), S.bf16_bits(Wk), S.bf16_bits(Wv), n_h, n_kv, d_h, t)
     assert np.array_equal(host_bits(out), ref)
+
+
+# ---------------------------------------------------------------------------------- AllToAll
+@pytest.mark.parametrize("t,rows,cols,split,concat,dtype", [
+    (4, 64, 256, 1, 0, "f32"), (4, 64, 256, 0, 1, "bf16"), (2, 32, 64, 0, 0, "f32"), (8, 64, 512, 1, 1, "bf16"),
+    (3, 9, 12, 1, 0, "f32"), (4, 8, 20, 0, 1, "bf16"), (8, 1024, 4096, 1, 0, "f32"),
+])
+def test_all_to_all_bit_exact(t, rows, cols, split, concat, dtype):
+    ins = _payload(t, rows, cols, dtype, seed=rows + cols + t)
+    ref = OC.all_to_all([host_bits(x) for x in ins], split_axis=split, concat_axis=concat)
+    d_in = [cuda(x) for x in ins]
+    d_out = [torch.empty(ref[0].shape, dtype=TD[dtype], device="cuda") for _ in range(t)]
+    tp.tp_all_to_all(d_in, d_out, rows, cols, split, concat, TPD[dtype], t)
+    torch.cuda.synchronize()
+    for j in range(t):
+        assert same_bits(host_bits(d_out[j]), ref[j]), f"shard {j}"
+
+
+def test_all_to_all_moves_the_sharded_dim():
+    # "Scaling Book 入门第 6 章", §6.4: AllToAll_{X,J}(A[I_X, J]) -> A[I, J_X]
+    t, I, J = 4, 64, 128
+    A = S.Draw(3).normal((I, J), 1.0, dtype=torch.float32)
+    ins = [cuda(b) for b in A.chunk(t, 0)]
+    outs = [torch.empty((I, J // t), device="cuda") for _ in range(t)]
+    tp.tp_all_to_all(ins, outs, I // t, J, 1, 0, tp.TP_F32, t)
+    torch.cuda.synchronize()
+    for j in range(t):
+        assert torch.equal(outs[j].cpu(), A[:, j * J // t:(j + 1) * J // t])

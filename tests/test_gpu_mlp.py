@@ -259,3 +259,33 @@ def test_llama70b_layer_sampled_rows():
         assert same_bits(host_bits(y[s]), host_bits(y[0]))
     # the MLP contribution alone, y - h1, against the oracle's
     assert_close(f64(y[0])[rows] - f64(h1[0])[rows], ref["mlp"], GEMM_TOL, "mlp part")
+
+
+# ---------------------------------------------------------------------------------- TP + SP MLP
+@pytest.mark.parametrize("N,h,F,t,act", [(512, 256, 1024, 4, tp.TP_ACT_GELU), (1024, 512, 2048, 4, tp.TP_ACT_SWIGLU),
+                                         (2048, 1024, 4096, 8, tp.TP_ACT_SWIGLU)])
+def test_sp_mlp_matches_oracle_and_tp_rows_bitwise(N, h, F, t, act):
+    d = S.Draw(N + t)
+    X = d.normal((N, h), 1.0)
+    wn = 2 * F // t if act == tp.TP_ACT_SWIGLU else F // t
+    w_in = d.normal((t, h, wn), 0.05)
+    w_down = d.normal((t, F // t, h), 0.05)
+    dX, dw_in, dw_down = cuda(X), cuda(w_in), cuda(w_down)
+    x_shards = [cuda(xs) for xs in X.chunk(t, 0)]
+    z = torch.empty((t, N, F // t), dtype=torch.bfloat16, device="cuda")
+    out = [torch.empty((N // t, h), device="cuda") for _ in range(t)]
+    tp.tp_mlp_fwd_sp(x_shards, N, h, F, t, act, dw_in, dw_down, z, out)
+    # the column GEMM reading the shards in place gives the same activations as reading the gathered X
+    z_full = torch.empty_like(z)
+    tp.tp_column_linear(dX, N, h, F, t, act, dw_in, z_full)
+    ref_tp = [torch.empty((N // t, h), device="cuda") for _ in range(t)]
+    tp.tp_mlp_fwd(dX, N, h, F, t, act, dw_in, dw_down, torch.empty_like(z), None, tp.TP_OUT_RS, ref_tp)
+    torch.cuda.synchronize()
+    _status_ok()
+    assert torch.equal(z, z_full)
+    for r in range(t):
+        assert torch.equal(out[r], ref_tp[r]), f"shard {r}"
+    a = "swiglu" if act == tp.TP_ACT_SWIGLU else "gelu"
+    ref = OM.sp_mlp([f64(x) for x in X.chunk(t, 0)], [f64(w) for w in w_in], [f64(w) for w in w_down], a)
+    for r in range(t):
+        assert_close(f64(out[r]), ref[r], GEMM_TOL, f"SP shard {r}")

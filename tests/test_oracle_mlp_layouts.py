@@ -287,3 +287,23 @@ def test_layer_rows_are_independent():
     rows = np.array([3, 1])
     part = layer.layer_forward(X, sh["O"], sh["qkv"], sh["o"], sh["gu"], sh["d"], rows=rows)
     assert np.allclose(part["y"], full["y"][rows], rtol=1e-13, atol=1e-13)
+
+
+@pytest.mark.parametrize("act,t", [("gelu", 2), ("swiglu", 4)])
+def test_sp_mlp_equals_pure_tp_rows(act, t):
+    # "张量并行与序列并行", §序列并行: TP+SP replaces the entry f by an AllGather and the exit g by a
+    # ReduceScatter along s; the result is the same tensor, each shard keeping its own block of tokens.
+    g = np.random.default_rng(11)
+    N, h, F = 8, 6, 8
+    X = g.standard_normal((N, h))
+    if act == "swiglu":
+        Wg, Wu = g.standard_normal((h, F)), g.standard_normal((h, F))
+        W_in, shards_in = np.concatenate([Wg, Wu], 1), list(layouts.shard_gate_up(Wg, Wu, t))
+    else:
+        W_in = g.standard_normal((h, F))
+        shards_in = list(layouts.shard_cols(W_in, t))
+    W_out = g.standard_normal((F, h))
+    Y = mlp.mlp_unsharded(X, W_in, W_out, act)
+    out = mlp.sp_mlp(np.split(X, t, axis=0), shards_in, list(layouts.shard_rows(W_out, t)), act)
+    assert len(out) == t and all(o.shape == (N // t, h) for o in out)
+    assert np.allclose(np.concatenate(out, 0), Y, rtol=1e-12, atol=1e-12)
