@@ -158,6 +158,12 @@ tp_status tp_all_to_all(const void* const* in, void* const* out, int64_t rows, i
  * input). Aligned; K and N must be multiples of 8. groups <= TP_MAX_SHARDS. */
 tp_status tp_grouped_gemm(int groups, const uint16_t* const* a, const uint16_t* const* b, void* const* c,
                           int64_t M, int64_t N, int64_t K, tp_act act, tp_dtype c_dtype, void* stream);
+/* Grouped GEMM with transposed operand storage (no activation): c[g] = op(a[g]) . op(b[g]), where
+ * op(a) = a [M, K] (trans_a = 0) or a holds A^T as [K, M] (trans_a = 1), and op(b) = b [K, N]
+ * (trans_b = 0) or b holds B^T as [N, K] (trans_b = 1). Row strides are the stored row lengths.
+ * Used by the backward pass for X^T dH, Z^T dY and dY W^T. M, N and K multiples of 8, aligned. */
+tp_status tp_grouped_gemm_t(int groups, const uint16_t* const* a, int trans_a, const uint16_t* const* b, int trans_b,
+                            void* const* c, int64_t M, int64_t N, int64_t K, tp_dtype c_dtype, void* stream);
 /* Column-parallel linear ([TPSP] §矩阵乘法的两种切法; [CH06] §6.7): y[r] = act(x . w[r]) for every
  * shard r, from the full x [N, k] (shared by all shards) and the stacked shards w [t][k][n/t]
  * ([t][k][2n/t] = [gate_r | up_r] for SWIGLU, as written by tp_shard_gate_up). y is stacked
@@ -200,6 +206,21 @@ tp_status tp_row_linear_reduce(const uint16_t* x, int64_t N, int64_t k, int64_t 
 tp_status tp_mlp_fwd(const uint16_t* x, int64_t N, int64_t h, int64_t F, int t, tp_act act,
                      const uint16_t* w_in, const uint16_t* w_down, uint16_t* z_ws, float* const* partials,
                      tp_reduce mode, float* const* out, void* stream);
+
+/* Backward of the tensor-parallel MLP ([TPSP] §矩阵乘法的两种切法, backward bullets, and §f 和 g; [PFY]
+ * §Tensor Parallel, the gradient identities). dY is replicated, since g's backward is the identity:
+ *   dZ_r = dY W_down[r]^T;  dW_down[r] = Z_r^T dY;  dH_r = act'(H_r) * dZ_r (SwiGLU: dG = dZ*U*SiLU'(G),
+ *   dU = dZ*SiLU(G));  dW_in[r] = X^T dH_r;  dX = sum_r dH_r W_in[r]^T (f's backward: a ring AllReduce).
+ *   x, dy   bf16 [N, h];  w_in / w_down as in tp_mlp_fwd
+ *   h_pre   bf16 stacked [t][N][wn], the forward pre-activations H_r = X W_in[r] (wn = F/t, or 2F/t for
+ *           SwiGLU: [G | U]; e.g. from tp_column_linear with TP_ACT_NONE)
+ *   z       bf16 stacked [t][N][F/t], the forward activations Z_r
+ *   dz_ws   bf16 workspace [t][N][F/t];  dh_ws bf16 workspace [t][N][wn]
+ *   dw_in   fp32 stacked [t][h][wn];  dw_down fp32 stacked [t][F/t][h];  dx  t fp32 [N, h] (identical replicas)
+ * N, h and F/t multiples of 8; t | N. */
+tp_status tp_mlp_bwd(const uint16_t* x, const uint16_t* dy, int64_t N, int64_t h, int64_t F, int t, tp_act act,
+                     const uint16_t* w_in, const uint16_t* w_down, const uint16_t* h_pre, const uint16_t* z,
+                     uint16_t* dz_ws, uint16_t* dh_ws, float* dw_in, float* dw_down, float* const* dx, void* stream);
 
 /* ------------------------------------------------------------------------------------------------
  * Tensor + sequence parallelism ([TPSP] §序列并行：把剩下的激活也切开). In the replicated region each

@@ -107,3 +107,47 @@ def sp_mlp(x_shards, W_in_shards, W_out_shards, act: str, device_model: bool = F
     X = all_gather([np.asarray(x, dtype=np.float64) for x in x_shards], axis=0)[0]
     U = mlp_partials(X, W_in_shards, W_out_shards, act, device_model)
     return reduce_scatter_f64(U, axis=0)
+
+
+def act_derivative(H, act: str):
+    """d act / dH for the element-wise activations (SwiGLU is handled in mlp_backward):
+    GeLU' = Phi(x) + x phi(x); the tanh form differentiated as written; SiLU' = s (1 + x (1 - s))."""
+    x = np.asarray(H, dtype=np.float64)
+    if act == "none":
+        return np.ones_like(x)
+    if act == "gelu":
+        return 0.5 * (1.0 + erf(x / math.sqrt(2.0))) + x * np.exp(-0.5 * x * x) / math.sqrt(2.0 * math.pi)
+    if act == "gelu_tanh":
+        c, a = math.sqrt(2.0 / math.pi), 0.044715
+        th = np.tanh(c * (x + a * x ** 3))
+        return 0.5 * (1.0 + th) + 0.5 * x * (1.0 - th * th) * c * (1.0 + 3.0 * a * x * x)
+    raise ValueError(act)
+
+
+def mlp_backward(X, W_in_shards, W_out_shards, dY, act: str):
+    """Gradients of L = sum(Y * dY) for the tensor-parallel MLP, shard by shard
+    ("张量并行与序列并行", §矩阵乘法的两种切法: column-parallel backward needs an AllReduce of dX, and
+    row-parallel backward is local; pufanyi.com "ml-revisit-infra", §Tensor Parallel: dW_i = X^T dY_i,
+    dX = sum_i dY_i W_i^T, and for the row split dW_i = X_i^T dY, dX_i = dY W_i^T).
+    Returns dX (the sum over shards), its per-shard partials, and dW_in / dW_out per shard."""
+    X = np.asarray(X, dtype=np.float64)
+    dY = np.asarray(dY, dtype=np.float64)
+    out = {"dX_partials": [], "dW_in": [], "dW_out": []}
+    for W_in, W_out in zip(W_in_shards, W_out_shards):
+        W_in = np.asarray(W_in, dtype=np.float64)
+        W_out = np.asarray(W_out, dtype=np.float64)
+        H = X @ W_in
+        Z = activate(H, act)
+        dZ = dY @ W_out.T                       # row layer: input gradient, local
+        out["dW_out"].append(Z.T @ dY)          # row layer: weight gradient, local
+        if act == "swiglu":
+            f = H.shape[1] // 2
+            g, u = H[:, :f], H[:, f:]
+            s = 1.0 / (1.0 + np.exp(-g))
+            dH = np.concatenate([dZ * u * s * (1.0 + g * (1.0 - s)), dZ * g * s], axis=1)
+        else:
+            dH = dZ * act_derivative(H, act)
+        out["dW_in"].append(X.T @ dH)           # column layer: weight gradient, local
+        out["dX_partials"].append(dH @ W_in.T)  # column layer: input gradient, a partial sum
+    out["dX"] = sum(out["dX_partials"])
+    return out

@@ -36,7 +36,7 @@ EXPORTED = (
     "tp_num_sms", "tp_shard_cols", "tp_shard_rows", "tp_shard_gate_up", "tp_shard_qkv", "tp_reduce_scatter",
     "tp_all_gather", "tp_all_reduce", "tp_grouped_gemm", "tp_column_linear", "tp_row_linear", "tp_row_linear_reduce", "tp_mlp_fwd",
     "tp_sharded_matmul_ws_bytes", "tp_sharded_matmul", "tp_layer_fwd", "tp_mlp_fwd_noalloc",
-    "tp_column_linear_sp", "tp_mlp_fwd_sp", "tp_all_to_all",
+    "tp_column_linear_sp", "tp_mlp_fwd_sp", "tp_all_to_all", "tp_grouped_gemm_t", "tp_mlp_bwd",
 )
 
 _vp, _i64, _i32, _u64, _sz = C.c_void_p, C.c_int64, C.c_int, C.c_uint64, C.c_size_t
@@ -58,6 +58,8 @@ _SIGS = {
     "tp_all_reduce": (_i32, [_pp, _pp, _i64, _i64, _i32, _i32, _vp]),
     "tp_all_to_all": (_i32, [_pp, _pp, _i64, _i64, _i32, _i32, _i32, _i32, _vp]),
     "tp_grouped_gemm": (_i32, [_i32, _pp, _pp, _pp, _i64, _i64, _i64, _i32, _i32, _vp]),
+    "tp_grouped_gemm_t": (_i32, [_i32, _pp, _i32, _pp, _i32, _pp, _i64, _i64, _i64, _i32, _vp]),
+    "tp_mlp_bwd": (_i32, [_vp, _vp, _i64, _i64, _i64, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _pp, _vp]),
     "tp_column_linear": (_i32, [_vp, _i64, _i64, _i64, _i32, _i32, _vp, _vp, _vp]),
     "tp_row_linear": (_i32, [_vp, _i64, _i64, _i64, _i32, _vp, _pp, _vp]),
     "tp_row_linear_reduce": (_i32, [_vp, _i64, _i64, _i64, _i32, _vp, _i32, _i32, _pp, _pp, _vp]),
@@ -180,6 +182,16 @@ def tp_all_to_all(ins, outs, rows, cols, split_axis, concat_axis, dtype, t, stre
 # ---- GEMMs, MLP, cases, layer -----------------------------------------------------------------
 def tp_grouped_gemm(groups, a, b, c, M, N, K, act, c_dtype, stream=None):
     _call("tp_grouped_gemm", groups, _ptrs(a), _ptrs(b), _ptrs(c), M, N, K, act, c_dtype, _stream(stream))
+
+
+def tp_grouped_gemm_t(groups, a, trans_a, b, trans_b, c, M, N, K, c_dtype, stream=None):
+    _call("tp_grouped_gemm_t", groups, _ptrs(a), trans_a, _ptrs(b), trans_b, _ptrs(c), M, N, K, c_dtype,
+          _stream(stream))
+
+
+def tp_mlp_bwd(x, dy, N, h, F, t, act, w_in, w_down, h_pre, z, dz_ws, dh_ws, dw_in, dw_down, dx, stream=None):
+    _call("tp_mlp_bwd", _ptr(x), _ptr(dy), N, h, F, t, act, _ptr(w_in), _ptr(w_down), _ptr(h_pre), _ptr(z),
+          _ptr(dz_ws), _ptr(dh_ws), _ptr(dw_in), _ptr(dw_down), _ptrs(dx), _stream(stream))
 
 
 def tp_column_linear(x, N, k, n, t, act, w, y, stream=None):

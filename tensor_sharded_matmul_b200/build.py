@@ -23,7 +23,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libtp.so")
 
-SOURCES = ["status.cu", "layouts.cu", "collectives.cu", "gemm.cu", "api.cu", "noalloc.cu"]
+SOURCES = ["status.cu", "layouts.cu", "collectives.cu", "gemm.cu", "api.cu", "backward.cu", "noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
          "--expt-relaxed-constexpr", "-I", INCLUDE, "-I", CSRC]

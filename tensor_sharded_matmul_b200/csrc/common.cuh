@@ -65,6 +65,9 @@ struct GemmArgs {
   int a_slices;
   int64_t slice_rows;
   const uint16_t* a_slice[TP_MAX_SHARDS];
+  // Transposed storage: a_mn = A given as A^T [K][M] (row stride lda >= M); b_km = B given as
+  // B^T [N][K] (row stride ldb >= K).
+  bool a_mn, b_km;
 };
 tp_status grouped_gemm(const GemmArgs& g, cudaStream_t s);
 
@@ -83,6 +86,7 @@ struct RingGemmArgs {
   const void* resid;                 // RING_AR only, [M, N]
   tp_dtype resid_dtype;
   uint16_t* copy_bf16;               // RING_AR only, [M, N]
+  bool b_km;                         // B given as B^T [N][K] (row stride ldb >= K)
 };
 // True when every 128 x 256 output tile lies inside one chunk (the fused kernel's requirement).
 bool ring_gemm_fits(int64_t M, int64_t N, int t, int axis);

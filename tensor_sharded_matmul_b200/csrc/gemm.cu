@@ -52,7 +52,6 @@ constexpr uint32_t B_STAGE = BN * BK * 2;        // 32 KiB
 constexpr uint32_t B_BOX = 64 * BK * 2;          // one 64(N) x 64(K) box, 8 KiB
 constexpr uint32_t TMEM_COLS = 512;              // two 128 x 256 fp32 accumulators
 constexpr int RASTER_BAND = 16;                  // row-tiles per raster band
-constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, /*a_mn=*/false, /*b_mn=*/true);
 
 constexpr int GEMM_THREADS = 192;                // producer, MMA, 4 epilogue warps
 constexpr int RING_THREADS = 320;                // producer, MMA, 8 epilogue warps
@@ -64,7 +63,6 @@ constexpr int PAIR_STAGES = 6;
 constexpr uint32_t PAIR_A_STAGE = 128 * BK * 2;  // 16 KiB
 constexpr uint32_t PAIR_B_STAGE = 128 * BK * 2;  // 16 KiB: two 64-wide boxes
 constexpr size_t PAIR_SMEM = 1024 + PAIR_STAGES * (PAIR_A_STAGE + PAIR_B_STAGE) + 256;
-constexpr uint32_t IDESC_PAIR = idesc_bf16_f32(2 * BM, BN, /*a_mn=*/false, /*b_mn=*/true);
 constexpr size_t RING_SMEM = 1024 + STAGES * (A_STAGE + B_STAGE) + 8 * STAGING_PER_WARP + 256;
 constexpr size_t RING_PAIR_SMEM = 1024 + PAIR_STAGES * (PAIR_A_STAGE + PAIR_B_STAGE) + 8 * STAGING_PER_WARP + 256;
 
@@ -85,6 +83,9 @@ struct Ctl {
   uint32_t* status;
   unsigned long long budget;
   uint64_t b_policy;                       // L2 policy of the B (weight) loads
+  bool a_mn;                               // A given transposed: stored [K][M] (M contiguous)
+  bool b_km;                               // B given transposed: stored [N][K] (K contiguous)
+  uint32_t idesc;                          // instruction descriptor for these major-nesses
 };
 
 __device__ __forceinline__ bool wait_or_abort(const Ctl& c, uint32_t bar, uint32_t parity, uint32_t site) {
@@ -96,7 +97,7 @@ __device__ __forceinline__ bool wait_or_abort(const Ctl& c, uint32_t bar, uint32
 
 // Lays out barriers and the TMEM slot after the operand stages (and the staging area, if any).
 __device__ __forceinline__ Ctl setup_ctl(uint8_t* smem, uint32_t extra_bytes, uint32_t*& tmem_slot, uint32_t* status,
-                                         unsigned long long budget, bool keep_b) {
+                                         unsigned long long budget, bool keep_b, bool a_mn, bool b_km) {
   Ctl c;
   c.sA = smem;
   c.sB = smem + STAGES * A_STAGE;
@@ -111,6 +112,9 @@ __device__ __forceinline__ Ctl setup_ctl(uint8_t* smem, uint32_t extra_bytes, ui
   c.status = status;
   c.budget = budget;
   c.b_policy = keep_b ? l2_policy_evict_last() : l2_policy_evict_normal();
+  c.a_mn = a_mn;
+  c.b_km = b_km;
+  c.idesc = idesc_bf16_f32(BM, BN, a_mn, !b_km);
   return c;
 }
 
@@ -140,9 +144,16 @@ __device__ __forceinline__ bool produce_unit(const Ctl& c, Ring& r, const CUtens
     const uint32_t a_dst = smem_u32(c.sA + r.stage * A_STAGE);
     const uint32_t b_dst = smem_u32(c.sB + r.stage * B_STAGE);
     const int k0 = kb * BK;
-    tma_load_2d(a_dst, a, k0, m0, fb);
-    // B (the weights) is re-read by every row-tile: keep its lines in L2 longest
-    if (b2 != nullptr) {
+    if (c.a_mn) {                       // A^T [K][M]: two 64(M) x 64(K) boxes
+      tma_load_2d(a_dst, a, m0, k0, fb);
+      tma_load_2d(a_dst + B_BOX, a, m0 + 64, k0, fb);
+    } else {                            // A [M][K]: one 64(K) x 128(M) box
+      tma_load_2d(a_dst, a, k0, m0, fb);
+    }
+    // B (the weights) is re-read by every row-tile: the fused kernel keeps its lines in L2 longest
+    if (c.b_km) {                       // B^T [N][K]: one 64(K) x 256(N) box
+      tma_load_2d_hint(b_dst, b, k0, n0, fb, c.b_policy);
+    } else if (b2 != nullptr) {
       tma_load_2d_hint(b_dst + 0 * B_BOX, b, n0, k0, fb, c.b_policy);
       tma_load_2d_hint(b_dst + 1 * B_BOX, b, n0 + 64, k0, fb, c.b_policy);
       tma_load_2d_hint(b_dst + 2 * B_BOX, b2, n0, k0, fb, c.b_policy);
@@ -167,11 +178,13 @@ __device__ __forceinline__ bool mma_unit(const Ctl& c, Ring& r, uint32_t d_tmem,
     const uint32_t b_base = smem_u32(c.sB + r.stage * B_STAGE);
 #pragma unroll
     for (int k = 0; k < BK / 16; ++k) {
-      // K-major A: advance 16 elements = 32 bytes inside the swizzle atom.
-      const uint64_t ad = smem_desc_sw128(a_base + 32u * k, 16u, 1024u);
-      // MN-major B: advance 16 K rows = two 8-row groups of 1 KiB; 64-wide N blocks 8 KiB apart.
-      const uint64_t bd = smem_desc_sw128(b_base + 2048u * k, B_BOX, 1024u);
-      umma_bf16(d_tmem, ad, bd, IDESC, (kb | k) != 0 ? 1u : 0u);
+      // K-major: advance 16 elements = 32 bytes inside the swizzle atom (8-row atoms of 1 KiB).
+      // MN-major: advance 16 K rows = two 8-row groups of 1 KiB; 64-wide MN blocks 8 KiB apart.
+      const uint64_t ad = c.a_mn ? smem_desc_sw128(a_base + 2048u * k, B_BOX, 1024u)
+                                 : smem_desc_sw128(a_base + 32u * k, 16u, 1024u);
+      const uint64_t bd = c.b_km ? smem_desc_sw128(b_base + 32u * k, 16u, 1024u)
+                                 : smem_desc_sw128(b_base + 2048u * k, B_BOX, 1024u);
+      umma_bf16(d_tmem, ad, bd, c.idesc, (kb | k) != 0 ? 1u : 0u);
     }
     mma_issued = true;
     umma_commit(c.empty0 + 8 * r.stage);   // frees the stage once these MMAs have read it
@@ -258,6 +271,7 @@ struct GemmParams {
   // A given as row slices shared by all groups (the sequence-parallel entry: A = AllGather of t
   // row shards): row m of A is row m % slice_rows of ta[m / slice_rows]. 0 = one A per group.
   int a_slices, slice_rows;
+  bool a_mn, b_km;                  // A stored [K][M] / B stored [N][K] (transposed operands)
   uint32_t* status;
   unsigned long long budget;
 };
@@ -309,7 +323,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tcgen05_kernel(const __g
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint32_t* tmem_slot;
-  const Ctl c = setup_ctl(smem, 0, tmem_slot, p.status, p.budget, false);
+  const Ctl c = setup_ctl(smem, 0, tmem_slot, p.status, p.budget, false, p.a_mn, p.b_km);
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
 
@@ -415,6 +429,8 @@ struct PairCtl {
   unsigned long long budget;
   uint32_t rank;
   uint64_t b_policy;                         // L2 policy of the B (weight) loads
+  bool a_mn, b_km;                           // transposed operand storage (see Ctl)
+  uint32_t idesc;
 };
 
 struct PairRing {
@@ -427,7 +443,7 @@ struct PairRing {
 
 __device__ __forceinline__ PairCtl pair_setup(uint8_t* smem, uint32_t extra_bytes, uint32_t*& tmem_slot,
                                               uint32_t epilogue_warps_per_cta, uint32_t* status,
-                                              unsigned long long budget, bool keep_b) {
+                                              unsigned long long budget, bool keep_b, bool a_mn, bool b_km) {
   PairCtl c;
   c.sA = smem;
   c.sB = smem + PAIR_STAGES * PAIR_A_STAGE;
@@ -443,6 +459,9 @@ __device__ __forceinline__ PairCtl pair_setup(uint8_t* smem, uint32_t extra_byte
   c.budget = budget;
   c.rank = cluster_ctarank();
   c.b_policy = keep_b ? l2_policy_evict_last() : l2_policy_evict_normal();
+  c.a_mn = a_mn;
+  c.b_km = b_km;
+  c.idesc = idesc_bf16_f32(2 * BM, BN, a_mn, !b_km);
   if (threadIdx.x == 0) {
     for (int s = 0; s < PAIR_STAGES; ++s) {
       mbar_init(c.full0 + 8 * s, 1);
@@ -486,9 +505,18 @@ __device__ __forceinline__ bool pair_produce_unit(const PairCtl& c, PairRing& r,
     const uint32_t a_dst = smem_u32(c.sA + r.stage * PAIR_A_STAGE);
     const uint32_t b_dst = smem_u32(c.sB + r.stage * PAIR_B_STAGE);
     const int k0 = kb * BK;
-    tma_load_2d_pair(a_dst, ta, k0, m0, fb);
-    tma_load_2d_pair_hint(b_dst, tb, nb, k0, fb, c.b_policy);
-    tma_load_2d_pair_hint(b_dst + B_BOX, tb, nb + 64, k0, fb, c.b_policy);
+    if (c.a_mn) {                       // A^T [K][M]: two 64(M) x 64(K) boxes of this CTA's 128 rows
+      tma_load_2d_pair(a_dst, ta, m0, k0, fb);
+      tma_load_2d_pair(a_dst + B_BOX, ta, m0 + 64, k0, fb);
+    } else {
+      tma_load_2d_pair(a_dst, ta, k0, m0, fb);
+    }
+    if (c.b_km) {                       // B^T [N][K]: one 64(K) x 128(N) box of this CTA's columns
+      tma_load_2d_pair_hint(b_dst, tb, k0, nb, fb, c.b_policy);
+    } else {
+      tma_load_2d_pair_hint(b_dst, tb, nb, k0, fb, c.b_policy);
+      tma_load_2d_pair_hint(b_dst + B_BOX, tb, nb + 64, k0, fb, c.b_policy);
+    }
     r.advance();
   }
   return true;
@@ -518,9 +546,11 @@ __device__ __forceinline__ bool pair_mma_unit(const PairCtl& c, PairRing& r, uin
     const uint32_t b_base = smem_u32(c.sB + r.stage * PAIR_B_STAGE);
 #pragma unroll
     for (int k = 0; k < BK / 16; ++k) {
-      const uint64_t ad = smem_desc_sw128(a_base + 32u * k, 16u, 1024u);
-      const uint64_t bd = smem_desc_sw128(b_base + 2048u * k, B_BOX, 1024u);
-      umma_bf16_pair(d_tmem, ad, bd, IDESC_PAIR, (kb | k) != 0 ? 1u : 0u);
+      const uint64_t ad = c.a_mn ? smem_desc_sw128(a_base + 2048u * k, B_BOX, 1024u)
+                                 : smem_desc_sw128(a_base + 32u * k, 16u, 1024u);
+      const uint64_t bd = c.b_km ? smem_desc_sw128(b_base + 32u * k, 16u, 1024u)
+                                 : smem_desc_sw128(b_base + 2048u * k, B_BOX, 1024u);
+      umma_bf16_pair(d_tmem, ad, bd, c.idesc, (kb | k) != 0 ? 1u : 0u);
     }
     mma_issued = true;
     umma_commit_pair_mc(c.empty0 + 8 * r.stage, 0x3);   // frees the stage in both CTAs
@@ -581,7 +611,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     for (int g = 0; g < (p.a_slices ? p.a_slices : p.groups); ++g) prefetch_tmap(&p.ta[g]);
   }
   uint32_t* tmem_slot;
-  const PairCtl c = pair_setup(smem, 0, tmem_slot, 4, p.status, p.budget, false);
+  const PairCtl c = pair_setup(smem, 0, tmem_slot, 4, p.status, p.budget, false, p.a_mn, p.b_km);
   const uint32_t tmem_base = *tmem_slot;
   const int pair = blockIdx.x >> 1;
   const int pairs = gridDim.x >> 1;
@@ -661,6 +691,7 @@ struct RingGemmParams {
   int chunk;                        // rows (axis 0) or columns (axis 1) per chunk
   int chunk_tiles;                  // row-tiles (axis 0) or n-tiles (axis 1) per chunk
   int resid_bf16;
+  bool b_km;                        // B stored [N][K] (transposed)
   uint32_t* status;
   unsigned long long budget;
 };
@@ -735,7 +766,7 @@ __global__ void __launch_bounds__(RING_THREADS, 1) gemm_ring_kernel(const __grid
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint32_t* tmem_slot;
   // the fused kernel re-reads every shard's weight panels from each chunk: keep them in L2
-  const Ctl c = setup_ctl(smem, 8 * STAGING_PER_WARP, tmem_slot, p.status, p.budget, true);
+  const Ctl c = setup_ctl(smem, 8 * STAGING_PER_WARP, tmem_slot, p.status, p.budget, true, false, p.b_km);
   const uint32_t staging0 = smem_u32(smem + STAGES * (A_STAGE + B_STAGE));
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -863,7 +894,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(RING_THREADS, 1)
   }
   uint32_t* tmem_slot;
   // the fused kernel re-reads every shard's weight panels from each chunk: keep them in L2
-  const PairCtl c = pair_setup(smem, 8 * STAGING_PER_WARP, tmem_slot, 8, p.status, p.budget, true);
+  const PairCtl c = pair_setup(smem, 8 * STAGING_PER_WARP, tmem_slot, 8, p.status, p.budget, true, false, p.b_km);
   const uint32_t tmem_base = *tmem_slot;
   const uint32_t staging0 = smem_u32(smem + PAIR_STAGES * (PAIR_A_STAGE + PAIR_B_STAGE));
   const int pair = blockIdx.x >> 1;
@@ -1046,7 +1077,9 @@ tp_status grouped_gemm(const GemmArgs& g, cudaStream_t s) {
   if (g.M > INT32_MAX / 2 || g.N > INT32_MAX / 2 || g.K > INT32_MAX / 2) return fail(TP_ESHAPE, "GEMM size too large");
   const bool swiglu = g.epi == EPI_SWIGLU;
   if (g.K % 8 || g.N % 8 || g.lda % 8 || g.ldb % 8) return fail(TP_EALIGN, "K, N and row strides must be multiples of 8");
-  if (g.lda < g.K || g.ldb < (swiglu ? 2 * g.N : g.N)) return fail(TP_ESHAPE, "row stride shorter than the row");
+  if (g.M % 8 && g.a_mn) return fail(TP_EALIGN, "M must be a multiple of 8 for a transposed A");
+  if (g.lda < (g.a_mn ? g.M : g.K) || g.ldb < (g.b_km ? g.K : (swiglu ? 2 * g.N : g.N)))
+    return fail(TP_ESHAPE, "row stride shorter than the row");
   for (int i = 0; i < g.groups; ++i) {
     if ((!g.a_slices && g.a[i] == nullptr) || g.b[i] == nullptr || g.c[i] == nullptr) return fail(TP_EINVAL, "null GEMM operand %d", i);
     if ((!g.a_slices && !aligned16(g.a[i])) || !aligned16(g.b[i]) || !aligned16(g.c[i]))
@@ -1056,6 +1089,8 @@ tp_status grouped_gemm(const GemmArgs& g, cudaStream_t s) {
   std::memset(&p, 0, sizeof(p));
   const int tile_n = swiglu ? BN / 2 : BN;
   const bool pair = g.M >= 2 * BM && (g.a_slices == 0 || g.slice_rows % (2 * BM) == 0);
+  if (g.a_slices && g.a_mn) return fail(TP_EUNSUPPORTED, "row slices of a transposed A are not supported");
+  if (swiglu && g.b_km) return fail(TP_EUNSUPPORTED, "SwiGLU needs B as [K][2N]");
   if (g.a_slices) {
     if (g.a_slices > TP_MAX_SHARDS || g.slice_rows <= 0 || g.slice_rows % BM != 0 || g.slice_rows * g.a_slices != g.M)
       return fail(TP_ESHAPE, "A row slices must tile M in multiples of %d rows", BM);
@@ -1069,10 +1104,13 @@ tp_status grouped_gemm(const GemmArgs& g, cudaStream_t s) {
     p.slice_rows = static_cast<int>(g.slice_rows);
   }
   for (int i = 0; i < g.groups; ++i) {
-    if (!g.a_slices && !encode_bf16_2d(&p.ta[i], g.a[i], g.K, g.M, g.lda, BK, BM))
-      return fail(TP_ECUDA, "cannot encode the TMA descriptor of A[%d]", i);
-    if (!encode_bf16_2d(&p.tb[i], g.b[i], g.N, g.K, g.ldb, 64, BK))
-      return fail(TP_ECUDA, "cannot encode the TMA descriptor of B[%d]", i);
+    const bool a_ok = g.a_slices ? true
+                      : g.a_mn ? encode_bf16_2d(&p.ta[i], g.a[i], g.M, g.K, g.lda, 64, BK)
+                               : encode_bf16_2d(&p.ta[i], g.a[i], g.K, g.M, g.lda, BK, BM);
+    if (!a_ok) return fail(TP_ECUDA, "cannot encode the TMA descriptor of A[%d]", i);
+    const bool b_ok = g.b_km ? encode_bf16_2d(&p.tb[i], g.b[i], g.K, g.N, g.ldb, BK, pair ? 128 : BN)
+                             : encode_bf16_2d(&p.tb[i], g.b[i], g.N, g.K, g.ldb, 64, BK);
+    if (!b_ok) return fail(TP_ECUDA, "cannot encode the TMA descriptor of B[%d]", i);
     if (swiglu && !encode_bf16_2d(&p.tb2[i], g.b[i] + g.N, g.N, g.K, g.ldb, 64, BK))
       return fail(TP_ECUDA, "cannot encode the TMA descriptor of the up half of B[%d]", i);
     p.c[i] = g.c[i];
@@ -1080,6 +1118,8 @@ tp_status grouped_gemm(const GemmArgs& g, cudaStream_t s) {
   p.M = static_cast<int>(g.M);
   p.N = static_cast<int>(g.N);
   p.K = static_cast<int>(g.K);
+  p.a_mn = g.a_mn;
+  p.b_km = g.b_km;
   p.tiles_m = static_cast<int>((g.M + BM - 1) / BM);
   p.tiles_n = static_cast<int>((g.N + tile_n - 1) / tile_n);
   p.groups = g.groups;
@@ -1124,19 +1164,24 @@ tp_status ring_gemm(const RingGemmArgs& g, cudaStream_t s) {
   const int axis = g.op == RING_AR ? 0 : g.axis;
   if (!ring_gemm_fits(g.M, g.N, g.t, axis)) return fail(TP_EUNSUPPORTED, "chunks do not align with 128 x 256 tiles");
   if (g.K % 8 || g.N % 8 || g.lda % 8 || g.ldb % 8) return fail(TP_EALIGN, "K, N and row strides must be multiples of 8");
-  if (g.lda < g.K || g.ldb < g.N) return fail(TP_ESHAPE, "row stride shorter than the row");
+  if (g.lda < g.K || g.ldb < (g.b_km ? g.K : g.N)) return fail(TP_ESHAPE, "row stride shorter than the row");
   if (tp_status st = check_operands(g.t, g.a, g.b, g.out)) return st;
   if ((g.resid && !aligned16(g.resid)) || (g.copy_bf16 && !aligned16(g.copy_bf16)))
     return fail(TP_EALIGN, "residual or bf16 copy not 16-byte aligned");
   RingGemmParams p;
   std::memset(&p, 0, sizeof(p));
+  const int axis0 = g.op == RING_AR ? 0 : g.axis;
+  const int64_t chunk0 = axis0 == 0 ? g.M / g.t : g.N / g.t;
+  const bool pair = axis0 == 0 ? chunk0 % (2 * BM) == 0 : g.M >= 2 * BM;
   for (int i = 0; i < g.t; ++i) {
     if (!encode_bf16_2d(&p.ta[i], g.a[i], g.K, g.M, g.lda, BK, BM))
       return fail(TP_ECUDA, "cannot encode the TMA descriptor of A[%d]", i);
-    if (!encode_bf16_2d(&p.tb[i], g.b[i], g.N, g.K, g.ldb, 64, BK))
-      return fail(TP_ECUDA, "cannot encode the TMA descriptor of B[%d]", i);
+    const bool b_ok = g.b_km ? encode_bf16_2d(&p.tb[i], g.b[i], g.K, g.N, g.ldb, BK, pair ? 128 : BN)
+                             : encode_bf16_2d(&p.tb[i], g.b[i], g.N, g.K, g.ldb, 64, BK);
+    if (!b_ok) return fail(TP_ECUDA, "cannot encode the TMA descriptor of B[%d]", i);
     p.out[i] = g.out[i];
   }
+  p.b_km = g.b_km;
   p.resid = g.op == RING_AR ? g.resid : nullptr;
   p.resid_bf16 = g.resid_dtype == TP_BF16;
   p.copy_bf16 = g.op == RING_AR ? g.copy_bf16 : nullptr;
@@ -1146,7 +1191,6 @@ tp_status ring_gemm(const RingGemmArgs& g, cudaStream_t s) {
   p.axis = axis;
   p.chunk = static_cast<int>(axis == 0 ? g.M / g.t : g.N / g.t);
   // CTA pairs when every chunk is a whole number of 256-row (axis 0) or 256-column (axis 1) tiles
-  const bool pair = axis == 0 ? p.chunk % (2 * BM) == 0 : g.M >= 2 * BM;
   p.chunk_tiles = axis == 0 ? p.chunk / (pair ? 2 * BM : BM) : p.chunk / BN;
   p.tiles_m = static_cast<int>(g.M / BM);
   p.tiles_n = static_cast<int>((g.N + BN - 1) / BN);

@@ -307,3 +307,54 @@ def test_sp_mlp_equals_pure_tp_rows(act, t):
     out = mlp.sp_mlp(np.split(X, t, axis=0), shards_in, list(layouts.shard_rows(W_out, t)), act)
     assert len(out) == t and all(o.shape == (N // t, h) for o in out)
     assert np.allclose(np.concatenate(out, 0), Y, rtol=1e-12, atol=1e-12)
+
+
+# ------------------------------------------------------------------------------------ backward
+@pytest.mark.parametrize("act,t", [("gelu", 2), ("gelu_tanh", 2), ("swiglu", 2), ("none", 4)])
+def test_mlp_backward_against_finite_differences(act, t):
+    # Central differences of L(X, W) = sum(MLP(X) * dY) pin every gradient formula independently.
+    g = np.random.default_rng(21)
+    N, h, F = 3, 4, 8
+    X, dY = g.standard_normal((N, h)), g.standard_normal((N, h))
+    if act == "swiglu":
+        Wg, Wu = g.standard_normal((h, F)) * 0.5, g.standard_normal((h, F)) * 0.5
+        W_in, shards_in = np.concatenate([Wg, Wu], 1), list(layouts.shard_gate_up(Wg, Wu, t))
+    else:
+        W_in = g.standard_normal((h, F)) * 0.5
+        shards_in = list(layouts.shard_cols(W_in, t))
+    W_out = g.standard_normal((F, h)) * 0.5
+    shards_out = list(layouts.shard_rows(W_out, t))
+    grads = mlp.mlp_backward(X, shards_in, shards_out, dY, act)
+    loss = lambda X_, Win_, Wout_: float(np.sum(mlp.mlp_unsharded(X_, Win_, Wout_, act) * dY))  # noqa: E731
+    eps = 1e-6
+
+    def num(f, A):
+        G = np.zeros_like(A)
+        for idx in np.ndindex(A.shape):
+            Ap, Am = A.copy(), A.copy()
+            Ap[idx] += eps
+            Am[idx] -= eps
+            G[idx] = (f(Ap) - f(Am)) / (2 * eps)
+        return G
+
+    assert np.allclose(grads["dX"], num(lambda A: loss(A, W_in, W_out), X), rtol=1e-5, atol=1e-6)
+    assert np.allclose(np.concatenate(grads["dW_out"], 0), num(lambda A: loss(X, W_in, A), W_out), rtol=1e-5, atol=1e-6)
+    dWin = num(lambda A: loss(X, A, W_out), W_in)
+    f = F // t
+    for r in range(t):
+        if act == "swiglu":     # shard r's block is [gate cols r | up cols r]
+            want = np.concatenate([dWin[:, r * f:(r + 1) * f], dWin[:, F + r * f:F + (r + 1) * f]], 1)
+        else:
+            want = dWin[:, r * f:(r + 1) * f]
+        assert np.allclose(grads["dW_in"][r], want, rtol=1e-5, atol=1e-6)
+
+
+def test_column_backward_needs_the_sum_over_shards():
+    # "张量并行与序列并行", §矩阵乘法的两种切法: each shard's dX is only a partial sum; one shard's alone is wrong.
+    g = np.random.default_rng(5)
+    X, dY = g.standard_normal((4, 6)), g.standard_normal((4, 6))
+    W_in, W_out = g.standard_normal((6, 8)), g.standard_normal((8, 6))
+    grads = mlp.mlp_backward(X, list(layouts.shard_cols(W_in, 2)), list(layouts.shard_rows(W_out, 2)), dY, "gelu")
+    full = mlp.mlp_backward(X, [W_in], [W_out], dY, "gelu")
+    assert np.allclose(grads["dX"], full["dX"], rtol=1e-12, atol=1e-12)
+    assert not np.allclose(grads["dX_partials"][0], full["dX"], rtol=1e-2, atol=1e-2)
