@@ -22,6 +22,10 @@
  *     elements) where a function says "aligned"; otherwise TP_EALIGN. A dimension that t must divide
  *     and does not gives TP_EDIVIS (nothing is padded).
  *   - Buffers must not overlap unless a function states otherwise.
+ *   - Empty inputs: a call whose token count / row count (or, for a GEMM or collective, any output
+ *     dimension) is zero returns TP_OK: t and the sizes are still checked, but no data pointer is
+ *     read and nothing is launched. A negative size, and an empty contraction (K, h or F of zero,
+ *     which would leave the output undefined rather than empty), give TP_EINVAL.
  *   - Device-side waits are bounded; a wait that runs out records TP_ETIMEOUT in the device status
  *     word (read it with tp_device_status) and the kernel returns without finishing its work.
  */
@@ -39,7 +43,7 @@ extern "C" {
 
 typedef enum {
   TP_OK = 0,
-  TP_EINVAL = 1,        /* null pointer, non-positive size, bad enum value */
+  TP_EINVAL = 1,        /* null pointer, negative size, empty contraction, bad enum value */
   TP_ESHAPE = 2,        /* sizes inconsistent with each other */
   TP_EDIVIS = 3,        /* t does not divide a dimension it must split */
   TP_EALIGN = 4,        /* pointer or row stride not 16-byte aligned */

@@ -135,9 +135,10 @@ tp_status tp_grouped_gemm(int groups, const uint16_t* const* a, const uint16_t* 
 tp_status tp_column_linear(const uint16_t* x, int64_t N, int64_t k, int64_t n, int t, tp_act act, const uint16_t* w,
                            uint16_t* y, void* stream) {
   if (!valid_t(t)) return fail(TP_EINVAL, "t=%d outside 1..%d", t, TP_MAX_SHARDS);
+  if (N < 0 || k <= 0 || n <= 0) return fail(TP_EINVAL, "negative size or empty contraction");
+  if (N == 0) return TP_OK;                              // no tokens: nothing to compute
   if (x == nullptr || w == nullptr || y == nullptr) return fail(TP_EINVAL, "null pointer");
   if (!valid_act(act)) return fail(TP_EINVAL, "bad activation");
-  if (N <= 0 || k <= 0 || n <= 0) return fail(TP_EINVAL, "non-positive size");
   if (n % t) return fail(TP_EDIVIS, "t=%d does not divide n=%lld", t, (long long)n);
   return column_gemm(x, N, k, n / t, t, act, w, y, static_cast<cudaStream_t>(stream));
 }
@@ -145,8 +146,9 @@ tp_status tp_column_linear(const uint16_t* x, int64_t N, int64_t k, int64_t n, i
 tp_status tp_row_linear(const uint16_t* x, int64_t N, int64_t k, int64_t n, int t, const uint16_t* w,
                         float* const* partials, void* stream) {
   if (!valid_t(t)) return fail(TP_EINVAL, "t=%d outside 1..%d", t, TP_MAX_SHARDS);
+  if (N < 0 || k <= 0 || n <= 0) return fail(TP_EINVAL, "negative size or empty contraction");
+  if (N == 0) return TP_OK;                              // no tokens: nothing to compute
   if (x == nullptr || w == nullptr || partials == nullptr) return fail(TP_EINVAL, "null pointer");
-  if (N <= 0 || k <= 0 || n <= 0) return fail(TP_EINVAL, "non-positive size");
   if (k % t) return fail(TP_EDIVIS, "t=%d does not divide k=%lld", t, (long long)k);
   return row_gemm(x, N, k / t, n, t, w, partials, static_cast<cudaStream_t>(stream));
 }
@@ -155,8 +157,9 @@ tp_status tp_row_linear_reduce(const uint16_t* x, int64_t N, int64_t k, int64_t 
                                tp_reduce mode, int axis, float* const* out, float* const* partials, void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (!valid_t(t)) return fail(TP_EINVAL, "t=%d outside 1..%d", t, TP_MAX_SHARDS);
+  if (N < 0 || k <= 0 || n <= 0) return fail(TP_EINVAL, "negative size or empty contraction");
+  if (N == 0) return TP_OK;                              // no tokens: nothing to compute
   if (x == nullptr || w == nullptr || out == nullptr) return fail(TP_EINVAL, "null pointer");
-  if (N <= 0 || k <= 0 || n <= 0) return fail(TP_EINVAL, "non-positive size");
   if (mode != TP_OUT_RS && mode != TP_OUT_AR && mode != TP_OUT_RS_AG) return fail(TP_EINVAL, "mode must reduce");
   if (axis != 0 && axis != 1) return fail(TP_EINVAL, "axis must be 0 or 1");
   if (mode != TP_OUT_RS) axis = 0;
@@ -177,12 +180,13 @@ tp_status tp_mlp_fwd(const uint16_t* x, int64_t N, int64_t h, int64_t F, int t, 
                      void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (!valid_t(t)) return fail(TP_EINVAL, "t=%d outside 1..%d", t, TP_MAX_SHARDS);
+  if (N < 0 || h <= 0 || F <= 0) return fail(TP_EINVAL, "negative size or empty hidden/F dimension");
+  if (N == 0) return TP_OK;                              // no tokens: nothing to compute
   if (x == nullptr || w_in == nullptr || w_down == nullptr || z_ws == nullptr) return fail(TP_EINVAL, "null pointer");
   if (partials == nullptr && (mode == TP_OUT_PARTIALS || N % t != 0 || !ring_gemm_fits(N, h, t, 0)))
     return fail(TP_EINVAL, "null partials: needed unless the fused row GEMM + reduction applies (N/t a multiple of 128)");
   if (!valid_act(act)) return fail(TP_EINVAL, "bad activation");
   if (mode < TP_OUT_PARTIALS || mode > TP_OUT_RS_AG) return fail(TP_EINVAL, "bad reduce mode");
-  if (N <= 0 || h <= 0 || F <= 0) return fail(TP_EINVAL, "non-positive size");
   if (F % t) return fail(TP_EDIVIS, "t=%d does not divide F=%lld", t, (long long)F);
   if (mode != TP_OUT_PARTIALS && N % t) return fail(TP_EDIVIS, "t=%d does not divide the token count %lld", t, (long long)N);
   const int64_t f = F / t;
@@ -199,9 +203,10 @@ tp_status tp_mlp_fwd(const uint16_t* x, int64_t N, int64_t h, int64_t F, int t, 
 tp_status tp_column_linear_sp(const uint16_t* const* x, int64_t N, int64_t k, int64_t n, int t, tp_act act,
                               const uint16_t* w, uint16_t* y, void* stream) {
   if (!valid_t(t)) return fail(TP_EINVAL, "t=%d outside 1..%d", t, TP_MAX_SHARDS);
+  if (N < 0 || k <= 0 || n <= 0) return fail(TP_EINVAL, "negative size or empty contraction");
+  if (N == 0) return TP_OK;                              // no tokens: nothing to compute
   if (x == nullptr || w == nullptr || y == nullptr) return fail(TP_EINVAL, "null pointer");
   if (!valid_act(act)) return fail(TP_EINVAL, "bad activation");
-  if (N <= 0 || k <= 0 || n <= 0) return fail(TP_EINVAL, "non-positive size");
   if (n % t || N % t) return fail(TP_EDIVIS, "t=%d does not divide n or the token count", t);
   if ((N / t) % 128) return fail(TP_EUNSUPPORTED, "token shards must be multiples of 128 rows");
   const int64_t n_shard = n / t;
@@ -222,6 +227,8 @@ tp_status tp_mlp_fwd_sp(const uint16_t* const* x, int64_t N, int64_t h, int64_t 
                         void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (!valid_t(t)) return fail(TP_EINVAL, "t=%d outside 1..%d", t, TP_MAX_SHARDS);
+  if (N < 0 || h <= 0 || F <= 0) return fail(TP_EINVAL, "negative size or empty hidden/F dimension");
+  if (N == 0) return TP_OK;                              // no tokens: nothing to compute
   if (x == nullptr || w_in == nullptr || w_down == nullptr || z_ws == nullptr || out == nullptr)
     return fail(TP_EINVAL, "null pointer");
   if (F % t) return fail(TP_EDIVIS, "t=%d does not divide F=%lld", t, (long long)F);
@@ -247,9 +254,10 @@ tp_status tp_sharded_matmul(int case_id, int strategy, const uint16_t* const* x,
                             void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (!valid_t(t)) return fail(TP_EINVAL, "t=%d outside 1..%d", t, TP_MAX_SHARDS);
+  if (B < 0 || D <= 0 || F <= 0) return fail(TP_EINVAL, "negative size or empty contraction");
+  if (B == 0) return TP_OK;                              // no rows: nothing to compute
   if (x == nullptr || w == nullptr || c == nullptr) return fail(TP_EINVAL, "null pointer array");
   if (!valid_dtype(c_dtype)) return fail(TP_EINVAL, "bad dtype");
-  if (B <= 0 || D <= 0 || F <= 0) return fail(TP_EINVAL, "non-positive size");
   for (int i = 0; i < t; ++i)
     if (x[i] == nullptr || w[i] == nullptr || c[i] == nullptr) return fail(TP_EINVAL, "null shard pointer %d", i);
   const size_t need = tp_sharded_matmul_ws_bytes(case_id, strategy, B, D, F, t);
@@ -350,9 +358,10 @@ tp_status tp_layer_fwd(const uint16_t* x, const uint16_t* const* o, int64_t N, i
                        float* const* partials, float* const* y, void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (!valid_t(t)) return fail(TP_EINVAL, "t=%d outside 1..%d", t, TP_MAX_SHARDS);
+  if (N < 0 || h <= 0 || F <= 0 || n_h <= 0 || n_kv <= 0 || d_h <= 0) return fail(TP_EINVAL, "non-positive size");
+  if (N == 0) return TP_OK;                              // no tokens: nothing to compute
   if (!x || !o || !w_qkv || !w_o || !w_gu || !w_down || !qkv_out || !h1 || !h1_bf16 || !z_ws || !y)
     return fail(TP_EINVAL, "null pointer");
-  if (N <= 0 || h <= 0 || F <= 0 || n_h <= 0 || n_kv <= 0 || d_h <= 0) return fail(TP_EINVAL, "non-positive size");
   if (n_h % t || n_h % n_kv || (t <= n_kv ? n_kv % t != 0 : t % n_kv != 0))
     return fail(TP_EDIVIS, "head counts n_h=%d n_kv=%d do not split over t=%d", n_h, n_kv, t);
   if (F % t || N % t) return fail(TP_EDIVIS, "t=%d does not divide F or the token count", t);

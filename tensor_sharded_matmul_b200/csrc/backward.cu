@@ -131,10 +131,11 @@ tp_status tp_mlp_bwd(const uint16_t* x, const uint16_t* dy, int64_t N, int64_t h
                      uint16_t* dz_ws, uint16_t* dh_ws, float* dw_in, float* dw_down, float* const* dx, void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (!valid_t(t)) return fail(TP_EINVAL, "t=%d outside 1..%d", t, TP_MAX_SHARDS);
+  if (N < 0 || h <= 0 || F <= 0) return fail(TP_EINVAL, "negative size or empty hidden/F dimension");
+  if (N == 0) return TP_OK;                              // no tokens: nothing to compute
   if (!x || !dy || !w_in || !w_down || !h_pre || !z || !dz_ws || !dh_ws || !dw_in || !dw_down || !dx)
     return fail(TP_EINVAL, "null pointer");
   if (!valid_act(act)) return fail(TP_EINVAL, "bad activation");
-  if (N <= 0 || h <= 0 || F <= 0) return fail(TP_EINVAL, "non-positive size");
   if (F % t || N % t) return fail(TP_EDIVIS, "t=%d does not divide F or the token count", t);
   if (N % 8 || h % 8 || (F / t) % 8) return fail(TP_EALIGN, "token count, h and F/t must be multiples of 8");
   for (int r = 0; r < t; ++r)

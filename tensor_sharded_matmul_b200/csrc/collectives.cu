@@ -257,7 +257,8 @@ void dispatch_reduce(const RingParams& p, tp_dtype din, tp_dtype dout, int block
 
 tp_status ring_collective(const RingArgs& a, cudaStream_t stream) {
   if (!valid_t(a.t)) return fail(TP_EINVAL, "t=%d outside 1..%d", a.t, TP_MAX_SHARDS);
-  if (a.rows <= 0 || a.cols <= 0) return fail(TP_EINVAL, "non-positive size");
+  if (a.rows < 0 || a.cols < 0) return fail(TP_EINVAL, "negative size");
+  if (a.rows == 0 || a.cols == 0) return TP_OK;         // empty buffers: nothing to move
   if (a.axis != 0 && a.axis != 1) return fail(TP_EINVAL, "axis must be 0 or 1");
   if ((a.in_dtype != TP_F32 && a.in_dtype != TP_BF16) || (a.out_dtype != TP_F32 && a.out_dtype != TP_BF16))
     return fail(TP_EINVAL, "bad dtype");
@@ -326,7 +327,8 @@ tp_status all_to_all(const void* const* in, void* const* out, int64_t rows, int6
                      tp_dtype dtype, int t, cudaStream_t stream) {
   if (in == nullptr || out == nullptr) return fail(TP_EINVAL, "null pointer array");
   if (!valid_t(t)) return fail(TP_EINVAL, "t=%d outside 1..%d", t, TP_MAX_SHARDS);
-  if (rows <= 0 || cols <= 0) return fail(TP_EINVAL, "non-positive size");
+  if (rows < 0 || cols < 0) return fail(TP_EINVAL, "negative size");
+  if (rows == 0 || cols == 0) return TP_OK;             // empty buffers: nothing to move
   if ((split != 0 && split != 1) || (concat != 0 && concat != 1)) return fail(TP_EINVAL, "axes must be 0 or 1");
   if (dtype != TP_F32 && dtype != TP_BF16) return fail(TP_EINVAL, "bad dtype");
   if (split == 0 ? rows % t : cols % t) return fail(TP_EDIVIS, "t=%d does not divide the split dimension", t);

@@ -1073,7 +1073,8 @@ tp_status check_operands(int n, const uint16_t* const* a, const uint16_t* const*
 
 tp_status grouped_gemm(const GemmArgs& g, cudaStream_t s) {
   if (g.groups < 1 || g.groups > TP_MAX_SHARDS) return fail(TP_EINVAL, "groups=%d outside 1..%d", g.groups, TP_MAX_SHARDS);
-  if (g.M <= 0 || g.N <= 0 || g.K <= 0) return fail(TP_EINVAL, "non-positive GEMM size");
+  if (g.M < 0 || g.N < 0 || g.K <= 0) return fail(TP_EINVAL, "negative GEMM size or empty contraction (K = 0)");
+  if (g.M == 0 || g.N == 0) return TP_OK;               // empty output: nothing to compute
   if (g.M > INT32_MAX / 2 || g.N > INT32_MAX / 2 || g.K > INT32_MAX / 2) return fail(TP_ESHAPE, "GEMM size too large");
   const bool swiglu = g.epi == EPI_SWIGLU;
   if (g.K % 8 || g.N % 8 || g.lda % 8 || g.ldb % 8) return fail(TP_EALIGN, "K, N and row strides must be multiples of 8");
@@ -1158,7 +1159,8 @@ bool ring_gemm_fits(int64_t M, int64_t N, int t, int axis) {
 
 tp_status ring_gemm(const RingGemmArgs& g, cudaStream_t s) {
   if (!valid_t(g.t)) return fail(TP_EINVAL, "t=%d outside 1..%d", g.t, TP_MAX_SHARDS);
-  if (g.M <= 0 || g.N <= 0 || g.K <= 0) return fail(TP_EINVAL, "non-positive GEMM size");
+  if (g.M < 0 || g.N < 0 || g.K <= 0) return fail(TP_EINVAL, "negative GEMM size or empty contraction (K = 0)");
+  if (g.M == 0 || g.N == 0) return TP_OK;               // empty output: nothing to compute
   if (g.M > INT32_MAX / 2 || g.N > INT32_MAX / 2 || g.K > INT32_MAX / 2) return fail(TP_ESHAPE, "GEMM size too large");
   if (g.op != RING_RS && g.op != RING_AR) return fail(TP_EINVAL, "fused GEMM reduces by RS or AR only");
   const int axis = g.op == RING_AR ? 0 : g.axis;

@@ -67,10 +67,10 @@ tp_status launch_segments(SegParams& p, cudaStream_t stream) {
     vec = aligned16(p.src[s]) && p.ld[s] % 8 == 0 && p.len[s] % 8 == 0;
     for (int r = 0; r < p.t && vec; ++r) vec = p.col0[s][r] % 8 == 0;
   }
+  const int64_t units = p.t * p.rows * (p.width / (vec ? 8 : 1));
+  if (units == 0) return TP_OK;                         // empty weight: nothing to copy
   const int sms = sm_count();
   if (sms <= 0) return fail(TP_ECUDA, "cannot query the SM count");
-  const int64_t units = p.t * p.rows * (p.width / (vec ? 8 : 1));
-  if (units == 0) return TP_OK;
   const int64_t want = (units + 255) / 256;
   const int blocks = static_cast<int>(want < static_cast<int64_t>(sms) * 8 ? want : static_cast<int64_t>(sms) * 8);
   if (vec)
@@ -80,10 +80,13 @@ tp_status launch_segments(SegParams& p, cudaStream_t stream) {
   return check_launch("segment_copy_kernel");
 }
 
-tp_status common_checks(const void* out, int t, int64_t rows, int64_t cols) {
+// Sets *empty (and returns TP_OK) for a weight with no elements: nothing is read or launched then.
+tp_status common_checks(const void* out, int t, int64_t rows, int64_t cols, bool* empty) {
   if (!valid_t(t)) return fail(TP_EINVAL, "t=%d outside 1..%d", t, TP_MAX_SHARDS);
+  if (rows < 0 || cols < 0) return fail(TP_EINVAL, "negative size %lld x %lld", (long long)rows, (long long)cols);
+  *empty = rows == 0 || cols == 0;
+  if (*empty) return TP_OK;
   if (out == nullptr) return fail(TP_EINVAL, "null output");
-  if (rows <= 0 || cols <= 0) return fail(TP_EINVAL, "non-positive size %lld x %lld", (long long)rows, (long long)cols);
   return TP_OK;
 }
 
@@ -95,7 +98,9 @@ using namespace tpx;
 extern "C" {
 
 tp_status tp_shard_cols(const uint16_t* w, int64_t ld, int64_t K, int64_t N, int t, uint16_t* out, void* stream) {
-  if (tp_status s = common_checks(out, t, K, N)) return s;
+  bool empty = false;
+  if (tp_status s = common_checks(out, t, K, N, &empty)) return s;
+  if (empty) return TP_OK;
   if (w == nullptr || ld < N) return fail(TP_EINVAL, "null weight or row stride %lld < %lld", (long long)ld, (long long)N);
   if (N % t) return fail(TP_EDIVIS, "t=%d does not divide N=%lld", t, (long long)N);
   SegParams p;
@@ -107,7 +112,9 @@ tp_status tp_shard_cols(const uint16_t* w, int64_t ld, int64_t K, int64_t N, int
 }
 
 tp_status tp_shard_rows(const uint16_t* w, int64_t ld, int64_t K, int64_t N, int t, uint16_t* out, void* stream) {
-  if (tp_status s = common_checks(out, t, K, N)) return s;
+  bool empty = false;
+  if (tp_status s = common_checks(out, t, K, N, &empty)) return s;
+  if (empty) return TP_OK;
   if (w == nullptr || ld < N) return fail(TP_EINVAL, "null weight or row stride %lld < %lld", (long long)ld, (long long)N);
   if (K % t) return fail(TP_EDIVIS, "t=%d does not divide K=%lld", t, (long long)K);
   SegParams p;
@@ -120,7 +127,9 @@ tp_status tp_shard_rows(const uint16_t* w, int64_t ld, int64_t K, int64_t N, int
 
 tp_status tp_shard_gate_up(const uint16_t* w_gate, int64_t ld_g, const uint16_t* w_up, int64_t ld_u, int64_t h,
                            int64_t F, int t, uint16_t* out, void* stream) {
-  if (tp_status s = common_checks(out, t, h, F)) return s;
+  bool empty = false;
+  if (tp_status s = common_checks(out, t, h, F, &empty)) return s;
+  if (empty) return TP_OK;
   if (w_gate == nullptr || w_up == nullptr || ld_g < F || ld_u < F) return fail(TP_EINVAL, "null weight or short row stride");
   if (F % t) return fail(TP_EDIVIS, "t=%d does not divide F=%lld", t, (long long)F);
   SegParams p;
@@ -138,7 +147,9 @@ tp_status tp_shard_gate_up(const uint16_t* w_gate, int64_t ld_g, const uint16_t*
 
 tp_status tp_shard_qkv(const uint16_t* w_q, int64_t ld_q, const uint16_t* w_k, int64_t ld_k, const uint16_t* w_v,
                        int64_t ld_v, int64_t h, int n_h, int n_kv, int d_h, int t, uint16_t* out, void* stream) {
-  if (tp_status s = common_checks(out, t, h, 1)) return s;
+  bool empty = false;
+  if (tp_status s = common_checks(out, t, h, 1, &empty)) return s;
+  if (empty) return TP_OK;
   if (w_q == nullptr || w_k == nullptr || w_v == nullptr) return fail(TP_EINVAL, "null QKV weight");
   if (n_h <= 0 || n_kv <= 0 || d_h <= 0) return fail(TP_EINVAL, "non-positive head counts");
   if (ld_q < int64_t(n_h) * d_h || ld_k < int64_t(n_kv) * d_h || ld_v < int64_t(n_kv) * d_h)

@@ -65,7 +65,8 @@ extern "C" tp_status tp_mlp_fwd_noalloc(const uint16_t* x, int64_t N, int64_t h,
                                         float* const* out, void* stream) {
   if (!valid_t(t)) return fail(TP_EINVAL, "t=%d outside 1..%d", t, TP_MAX_SHARDS);
   if (out == nullptr) return fail(TP_EINVAL, "null output array");
-  if (N <= 0 || h <= 0 || F <= 0) return fail(TP_EINVAL, "non-positive size");
+  if (N < 0 || h <= 0 || F <= 0) return fail(TP_EINVAL, "negative size or empty hidden/F dimension");
+  if (N == 0) return TP_OK;                              // no tokens: nothing to compute
   if (mode < TP_OUT_PARTIALS || mode > TP_OUT_RS_AG) return fail(TP_EINVAL, "bad reduce mode");
   // Scratch: Z as bf16 [t][N][F/t], plus t fp32 [N, h] partials unless the caller's outputs hold them.
   const size_t z_bytes = round256(size_t(N) * size_t(F) * 2);

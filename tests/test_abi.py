@@ -63,7 +63,7 @@ def test_collectives_validate_before_launch():
     _expect(tp.TP_EDIVIS, tp.tp_all_gather, [FAKE] * 3, [FAKE] * 3, 16, 16, 1, tp.TP_BF16, 3, 0)
     _expect(tp.TP_EINVAL, tp.tp_all_reduce, [FAKE, 0], [FAKE, FAKE], 16, 16, tp.TP_F32, 2, 0)
     _expect(tp.TP_EINVAL, tp.tp_reduce_scatter, [FAKE] * 2, [FAKE] * 2, 16, 16, 2, tp.TP_F32, 2, 0)
-    _expect(tp.TP_EINVAL, tp.tp_reduce_scatter, [FAKE] * 2, [FAKE] * 2, 0, 16, 0, tp.TP_F32, 2, 0)
+    _expect(tp.TP_EINVAL, tp.tp_reduce_scatter, [FAKE] * 2, [FAKE] * 2, -2, 16, 0, tp.TP_F32, 2, 0)
 
 
 def test_layouts_validate_before_launch():
@@ -108,3 +108,32 @@ def test_layer_validates_head_split():
     args = [FAKE, [FAKE] * 3, 96, 256, 8, 2, 32, 768, 3, FAKE, FAKE, FAKE, FAKE, FAKE, [FAKE] * 3, FAKE, FAKE,
             [FAKE] * 3, [FAKE] * 3, 0]
     _expect(tp.TP_EDIVIS, tp.tp_layer_fwd, *args)
+
+
+def test_empty_inputs_are_noops_without_a_gpu():
+    """A zero token/row count returns TP_OK having read no data pointer and launched nothing, which
+    is why these calls succeed on a host with no GPU (null data pointers included: an empty tensor
+    may have none). t and the sizes are still validated."""
+    E = [0, 0]
+    tp.tp_reduce_scatter(E, E, 0, 16, 0, tp.TP_F32, 2, 0)
+    tp.tp_all_gather(E, E, 16, 0, 1, tp.TP_BF16, 2, 0)
+    tp.tp_all_reduce(E, E, 0, 0, tp.TP_F32, 2, 0)
+    tp.tp_all_to_all(E, E, 0, 16, 0, 1, tp.TP_BF16, 2, 0)
+    tp.tp_shard_cols(0, 16, 0, 16, 2, FAKE, 0)
+    tp.tp_shard_gate_up(0, 16, 0, 16, 0, 16, 2, FAKE, 0)
+    tp.tp_grouped_gemm(2, E, E, E, 0, 64, 64, tp.TP_ACT_NONE, tp.TP_F32, 0)
+    tp.tp_grouped_gemm_t(2, E, 1, E, 1, E, 64, 0, 64, tp.TP_BF16, 0)
+    tp.tp_column_linear(0, 0, 256, 1024, 4, tp.TP_ACT_GELU, 0, 0, 0)
+    tp.tp_row_linear(0, 0, 1024, 256, 4, 0, [0] * 4, 0)
+    tp.tp_row_linear_reduce(0, 0, 1024, 256, 4, 0, tp.TP_OUT_AR, 0, [0] * 4, None, 0)
+    tp.tp_mlp_fwd(0, 0, 256, 1024, 4, tp.TP_ACT_SWIGLU, 0, 0, 0, None, tp.TP_OUT_RS, [0] * 4, 0)
+    tp.tp_mlp_fwd_noalloc(0, 0, 256, 1024, 4, tp.TP_ACT_GELU, 0, 0, tp.TP_OUT_AR, [0] * 4, 0)
+    tp.tp_mlp_fwd_sp([0] * 4, 0, 256, 1024, 4, tp.TP_ACT_GELU, 0, 0, 0, [0] * 4, 0)
+    tp.tp_mlp_bwd(0, 0, 0, 256, 1024, 4, tp.TP_ACT_GELU, 0, 0, 0, 0, 0, 0, 0, 0, [0] * 4, 0)
+    tp.tp_sharded_matmul(3, 0, [0] * 4, [0] * 4, 0, 64, 64, 4, [0] * 4, tp.TP_F32, 0, 0, 0)
+    tp.tp_layer_fwd(0, [0] * 2, 0, 256, 8, 2, 32, 768, 2, 0, 0, 0, 0, 0, [0] * 2, 0, 0, None, [0] * 2, 0)
+    # still validated: t, negative sizes, empty contractions
+    _expect(tp.TP_EINVAL, tp.tp_column_linear, 0, 0, 256, 1024, 0, tp.TP_ACT_GELU, 0, 0, 0)
+    _expect(tp.TP_EINVAL, tp.tp_column_linear, 0, -1, 256, 1024, 4, tp.TP_ACT_GELU, 0, 0, 0)
+    _expect(tp.TP_EINVAL, tp.tp_grouped_gemm, 1, [FAKE], [FAKE], [FAKE], 64, 64, 0, tp.TP_ACT_NONE, tp.TP_F32, 0)
+    _expect(tp.TP_EINVAL, tp.tp_mlp_fwd, 0, 0, 0, 1024, 4, tp.TP_ACT_GELU, 0, 0, 0, None, tp.TP_OUT_RS, [0] * 4, 0)

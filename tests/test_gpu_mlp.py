@@ -289,3 +289,30 @@ def test_sp_mlp_matches_oracle_and_tp_rows_bitwise(N, h, F, t, act):
     ref = OM.sp_mlp([f64(x) for x in X.chunk(t, 0)], [f64(w) for w in w_in], [f64(w) for w in w_down], a)
     for r in range(t):
         assert_close(f64(out[r]), ref[r], GEMM_TOL, f"SP shard {r}")
+
+
+# ---------------------------------------------------------------------------------- empty inputs
+def test_empty_token_count_is_a_noop_then_a_normal_call_matches():
+    """N = 0 launches nothing and leaves the output untouched; the next non-empty call on the same
+    stream is unaffected (no error state, no device status)."""
+    N, h, F, t = 64, 256, 1024, 4
+    X, A, B = S.tiny_mlp(seed=3)
+    dX = cuda(X)
+    w_in = torch.empty((t, h, F // t), dtype=torch.bfloat16, device="cuda")
+    w_down = torch.empty((t, F // t, h), dtype=torch.bfloat16, device="cuda")
+    tp.tp_shard_cols(cuda(A), F, h, F, t, w_in)
+    tp.tp_shard_rows(cuda(B), h, F, h, t, w_down)
+    empty_x = torch.empty((0, h), dtype=torch.bfloat16, device="cuda")
+    z0 = torch.empty((t, 0, F // t), dtype=torch.bfloat16, device="cuda")
+    sentinel = [torch.full((4, h), 7.0, device="cuda") for _ in range(t)]
+    tp.tp_mlp_fwd(empty_x, 0, h, F, t, tp.TP_ACT_GELU, w_in, w_down, z0, None, tp.TP_OUT_AR, sentinel)
+    tp.tp_all_reduce(sentinel, sentinel, 0, h, tp.TP_F32, t)
+    tp.tp_column_linear(empty_x, 0, h, F, t, tp.TP_ACT_GELU, w_in, z0)
+    torch.cuda.synchronize()
+    _status_ok()
+    for s in sentinel:
+        assert bool((s == 7.0).all())
+    _, _, out = _mlp_device(dX, w_in, w_down, N, h, F, t, tp.TP_ACT_GELU, tp.TP_OUT_AR)
+    Y = OM.mlp_unsharded(f64(X), f64(A), f64(B), "gelu")
+    for r in range(t):
+        assert_close(f64(out[r]), Y, GEMM_TOL, f"replica {r}")
