@@ -430,7 +430,8 @@ struct PairCtl {
   uint32_t rank;
   uint64_t b_policy;                         // L2 policy of the B (weight) loads
   bool a_mn, b_km;                           // transposed operand storage (see Ctl)
-  uint32_t idesc;
+  uint32_t idesc;                            // M=256, N=256
+  uint32_t idesc_half;                       // M=256, N=128 (half-width tiles)
 };
 
 struct PairRing {
@@ -462,6 +463,7 @@ __device__ __forceinline__ PairCtl pair_setup(uint8_t* smem, uint32_t extra_byte
   c.a_mn = a_mn;
   c.b_km = b_km;
   c.idesc = idesc_bf16_f32(2 * BM, BN, a_mn, !b_km);
+  c.idesc_half = idesc_bf16_f32(2 * BM, BN / 2, a_mn, !b_km);
   if (threadIdx.x == 0) {
     for (int s = 0; s < PAIR_STAGES; ++s) {
       mbar_init(c.full0 + 8 * s, 1);
@@ -494,13 +496,15 @@ __device__ __forceinline__ bool pair_fail(const PairCtl& c, uint32_t site) {
 }
 
 // Producer of one CTA: the num_kb k-blocks of one unit. m0 is this CTA's first row, nb its first
-// B column (two 64-wide boxes of `tb`).
+// B column: two 64-wide boxes of `tb` for a full tile, one for a half-width tile (wide == false,
+// B stored [K][N] only).
 __device__ __forceinline__ bool pair_produce_unit(const PairCtl& c, PairRing& r, const CUtensorMap* ta, int m0,
-                                                  const CUtensorMap* tb, int nb, int num_kb) {
+                                                  const CUtensorMap* tb, int nb, int num_kb, bool wide = true) {
+  const uint32_t tx = 2 * (PAIR_A_STAGE + (wide ? PAIR_B_STAGE : PAIR_B_STAGE / 2));
   for (int kb = 0; kb < num_kb; ++kb) {
     if (!mbar_wait_bounded(c.empty0 + 8 * r.stage, r.phase ^ 1u, c.budget, c.abort_flag))
       return pair_fail(c, WAIT_PRODUCER_EMPTY);
-    if (c.rank == 0) mbar_arrive_expect_tx(c.full0 + 8 * r.stage, 2 * (PAIR_A_STAGE + PAIR_B_STAGE));
+    if (c.rank == 0) mbar_arrive_expect_tx(c.full0 + 8 * r.stage, tx);
     const uint32_t fb = c.full0_leader + 8 * r.stage;
     const uint32_t a_dst = smem_u32(c.sA + r.stage * PAIR_A_STAGE);
     const uint32_t b_dst = smem_u32(c.sB + r.stage * PAIR_B_STAGE);
@@ -515,7 +519,7 @@ __device__ __forceinline__ bool pair_produce_unit(const PairCtl& c, PairRing& r,
       tma_load_2d_pair_hint(b_dst, tb, k0, nb, fb, c.b_policy);
     } else {
       tma_load_2d_pair_hint(b_dst, tb, nb, k0, fb, c.b_policy);
-      tma_load_2d_pair_hint(b_dst + B_BOX, tb, nb + 64, k0, fb, c.b_policy);
+      if (wide) tma_load_2d_pair_hint(b_dst + B_BOX, tb, nb + 64, k0, fb, c.b_policy);
     }
     r.advance();
   }
@@ -536,9 +540,10 @@ __device__ __forceinline__ bool pair_wait_acc_empty(const PairCtl& c, int acc, u
   return true;
 }
 
-// Leader's MMA thread: one unit's num_kb k-blocks into d_tmem (M=256 over the pair, N=256).
+// Leader's MMA thread: one unit's num_kb k-blocks into d_tmem (M=256 over the pair; N=256, or 128
+// with c.idesc_half).
 __device__ __forceinline__ bool pair_mma_unit(const PairCtl& c, PairRing& r, uint32_t d_tmem, int num_kb,
-                                              bool& mma_issued) {
+                                              bool& mma_issued, uint32_t idesc) {
   for (int kb = 0; kb < num_kb; ++kb) {
     if (!mbar_wait_bounded(c.full0 + 8 * r.stage, r.phase, c.budget, c.abort_flag)) return pair_fail(c, WAIT_MMA_FULL);
     tc_fence_after();
@@ -550,7 +555,7 @@ __device__ __forceinline__ bool pair_mma_unit(const PairCtl& c, PairRing& r, uin
                                  : smem_desc_sw128(a_base + 32u * k, 16u, 1024u);
       const uint64_t bd = c.b_km ? smem_desc_sw128(b_base + 32u * k, 16u, 1024u)
                                  : smem_desc_sw128(b_base + 2048u * k, B_BOX, 1024u);
-      umma_bf16_pair(d_tmem, ad, bd, c.idesc, (kb | k) != 0 ? 1u : 0u);
+      umma_bf16_pair(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
     }
     mma_issued = true;
     umma_commit_pair_mc(c.empty0 + 8 * r.stage, 0x3);   // frees the stage in both CTAs
@@ -643,7 +648,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
       uint32_t acc_phase = 0;
       for (int tile = pair; tile < num_tiles; tile += pairs) {
         if (!pair_wait_acc_empty(c, acc, acc_phase ^ 1u)) break;
-        if (!pair_mma_unit(c, r, tmem_base + static_cast<uint32_t>(acc * BN), p.num_kb, mma_issued)) break;
+        if (!pair_mma_unit(c, r, tmem_base + static_cast<uint32_t>(acc * BN), p.num_kb, mma_issued, c.idesc)) break;
         umma_commit_pair_mc(c.accf0 + 8 * acc, 0x3);   // both halves of the accumulator ready
         if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
       }
@@ -692,6 +697,12 @@ struct RingGemmParams {
   int chunk_tiles;                  // row-tiles (axis 0) or n-tiles (axis 1) per chunk
   int resid_bf16;
   bool b_km;                        // B stored [N][K] (transposed)
+  // CTA-pair kernel schedule: units [0, full_units) are 256 x 256 tiles in raster order; the
+  // remaining tiles are cut into two 256 x 128 halves each, units [full_units, num_units).
+  int full_units, num_units;
+  // AllReduce on CTA pairs: write replica 0 at the tile's end and copy it into the other t - 1
+  // replicas a slice at a time while the next tile's shards run.
+  bool defer_replicas;
   uint32_t* status;
   unsigned long long budget;
 };
@@ -711,7 +722,7 @@ __device__ __forceinline__ float4 ld_shared_v4(uint32_t addr) {
 // of bank conflicts. Each store instruction then covers four rows x 128 contiguous bytes (64 for bf16).
 template <bool OUT_BF16, bool AR>
 __device__ __forceinline__ void store_block32(const RingGemmParams& p, uint32_t stg, int lane, const float (&v)[32],
-                                              int row0, int col0, int c) {
+                                              int row0, int col0, int c, bool defer = false) {
 #pragma unroll
   for (int j = 0; j < 8; ++j)
     st_shared_v4(stg + lane * 128 + ((j ^ (lane & 7)) << 4), v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
@@ -737,12 +748,20 @@ __device__ __forceinline__ void store_block32(const RingGemmParams& p, uint32_t 
           }
           x.x = __fadd_rn(x.x, q.x); x.y = __fadd_rn(x.y, q.y); x.z = __fadd_rn(x.z, q.z); x.w = __fadd_rn(x.w, q.w);
         }
-        for (int s = 0; s < p.t; ++s) {
+        if (defer) {   // replica 0 only, kept in L2 for the copies that follow
           if constexpr (OUT_BF16)
-            st_cs_v2(static_cast<uint16_t*>(p.out[s]) + e, make_uint2(pack2(x.x, x.y), pack2(x.z, x.w)));
+            st_v2(static_cast<uint16_t*>(p.out[0]) + e, make_uint2(pack2(x.x, x.y), pack2(x.z, x.w)));
           else
-            st_cs_v4(static_cast<float*>(p.out[s]) + e, make_uint4(__float_as_uint(x.x), __float_as_uint(x.y),
-                                                                  __float_as_uint(x.z), __float_as_uint(x.w)));
+            st_v4(static_cast<float*>(p.out[0]) + e, make_uint4(__float_as_uint(x.x), __float_as_uint(x.y),
+                                                               __float_as_uint(x.z), __float_as_uint(x.w)));
+        } else {
+          for (int s = 0; s < p.t; ++s) {
+            if constexpr (OUT_BF16)
+              st_cs_v2(static_cast<uint16_t*>(p.out[s]) + e, make_uint2(pack2(x.x, x.y), pack2(x.z, x.w)));
+            else
+              st_cs_v4(static_cast<float*>(p.out[s]) + e, make_uint4(__float_as_uint(x.x), __float_as_uint(x.y),
+                                                                    __float_as_uint(x.z), __float_as_uint(x.w)));
+          }
         }
         if (p.copy_bf16 != nullptr) st_cs_v2(p.copy_bf16 + e, make_uint2(pack2(x.x, x.y), pack2(x.z, x.w)));
       } else {
@@ -758,6 +777,27 @@ __device__ __forceinline__ void store_block32(const RingGemmParams& p, uint32_t 
     }
   }
   __syncwarp();
+}
+
+// Deferred AllGather leg of the CTA-pair AllReduce: rows [r_begin, r_end) of one warp's region
+// (first row row0, first column col0, ncols columns) are copied from replica 0, which this warp
+// wrote, into replicas 1..t-1. Copying moves bits, so the replicas stay identical.
+template <bool OUT_BF16>
+__device__ __forceinline__ void copy_replica_rows(const RingGemmParams& p, int lane, int row0, int col0, int ncols,
+                                                  int r_begin, int r_end) {
+  constexpr int PER16 = OUT_BF16 ? 8 : 4;          // elements per 16-byte vector
+  constexpr int ESIZE = OUT_BF16 ? 2 : 4;
+  const int vec_per_row = ncols / PER16;
+  const int total = (r_end - r_begin) * vec_per_row;
+  for (int idx = lane; idx < total; idx += 32) {
+    const int row = row0 + r_begin + idx / vec_per_row;
+    const int col = col0 + (idx % vec_per_row) * PER16;
+    if (row < p.M && col < p.N) {
+      const int64_t off = (static_cast<int64_t>(row) * p.N + col) * ESIZE;
+      const uint4 v = ld_cg_v4(static_cast<const uint8_t*>(p.out[0]) + off);
+      for (int s = 1; s < p.t; ++s) st_cs_v4(static_cast<uint8_t*>(p.out[s]) + off, v);
+    }
+  }
 }
 
 template <bool OUT_BF16, bool AR>
@@ -875,8 +915,28 @@ __global__ void __launch_bounds__(RING_THREADS, 1) gemm_ring_kernel(const __grid
   teardown(c, warp, lane, last_phase, issued, mma_issued, tmem_base);
 }
 
+// Unit u of the CTA-pair fused kernel -> its tile's first row-tile, first column and width.
+__device__ __forceinline__ void ring_pair_unit(const RingGemmParams& p, int u, int tiles_m, int& mt, int& n0,
+                                               bool& wide) {
+  int tile = u, hsel = 0;
+  wide = u < p.full_units;
+  if (!wide) {
+    const int h = u - p.full_units;
+    tile = p.full_units + (h >> 1);
+    hsel = h & 1;
+  }
+  int nt;
+  raster_by_chunk(tile, tiles_m, p.tiles_n, p.axis, p.chunk_tiles, mt, nt);
+  n0 = nt * BN + hsel * (BN / 2);
+}
+
 // Fused row GEMM + ring reduction on CTA pairs: the same ring-ordered epilogue as
-// gemm_ring_kernel, each CTA summing and storing its own 128 rows of a 256 x 256 pair tile.
+// gemm_ring_kernel, each CTA summing and storing its own 128 rows of a 256-row pair tile.
+//  * Tiles are 256 x 256. When the last round of tiles would leave at least half of the pairs idle,
+//    those tiles are cut into 256 x 128 halves (MMA N = 128), so that round takes half the time.
+//  * AllReduce: at a tile's end only replica 0 is written; the copies into replicas 1..t-1 are
+//    spread over the next tile's t shard steps (1/t of the rows after each step), so the t-fold
+//    write traffic overlaps the tensor-core work instead of arriving as one burst per tile.
 template <bool OUT_BF16, bool AR>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(RING_THREADS, 1)
     gemm_ring_pair_kernel(const __grid_constant__ RingGemmParams p) {
@@ -900,22 +960,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(RING_THREADS, 1)
   const int pair = blockIdx.x >> 1;
   const int pairs = gridDim.x >> 1;
   const int tiles_m = (p.M + TILE_M - 1) / TILE_M;
-  const int num_tiles = tiles_m * p.tiles_n;
   bool mma_issued = false;
 
   if (warp == 0) {
     if (lane == 0) {
       PairRing r;
       bool ok = true;
-      for (int tile = pair; ok && tile < num_tiles; tile += pairs) {
-        int mt, nt;
-        raster_by_chunk(tile, tiles_m, p.tiles_n, p.axis, p.chunk_tiles, mt, nt);
-        const int ch = (p.axis == 0 ? mt * TILE_M : nt * BN) / p.chunk;
+      for (int u = pair; ok && u < p.num_units; u += pairs) {
+        int mt, n0;
+        bool wide;
+        ring_pair_unit(p, u, tiles_m, mt, n0, wide);
+        const int ch = (p.axis == 0 ? mt * TILE_M : n0) / p.chunk;
         const int m0 = mt * TILE_M + static_cast<int>(c.rank) * BM;
-        const int nb = nt * BN + static_cast<int>(c.rank) * 128;
+        const int nb = n0 + static_cast<int>(c.rank) * (wide ? 128 : 64);
         for (int j = 0; ok && j < t; ++j) {
           const int s = (ch + 1 + j) % t;              // ring order of this chunk
-          ok = pair_produce_unit(c, r, &p.ta[s], m0, &p.tb[s], nb, p.num_kb);
+          ok = pair_produce_unit(c, r, &p.ta[s], m0, &p.tb[s], nb, p.num_kb, wide);
         }
       }
     }
@@ -925,11 +985,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(RING_THREADS, 1)
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int tile = pair; ok && tile < num_tiles; tile += pairs) {
+      for (int u = pair; ok && u < p.num_units; u += pairs) {
+        const uint32_t idesc = u < p.full_units ? c.idesc : c.idesc_half;
         for (int j = 0; ok && j < t; ++j) {
           ok = pair_wait_acc_empty(c, acc, acc_phase ^ 1u);
           if (!ok) break;
-          ok = pair_mma_unit(c, r, tmem_base + static_cast<uint32_t>(acc * BN), p.num_kb, mma_issued);
+          ok = pair_mma_unit(c, r, tmem_base + static_cast<uint32_t>(acc * BN), p.num_kb, mma_issued, idesc);
           if (!ok) break;
           umma_commit_pair_mc(c.accf0 + 8 * acc, 0x3);
           if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
@@ -937,45 +998,60 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(RING_THREADS, 1)
       }
     }
   } else {
+    // warps 2..9: TMEM lane quadrant = warp % 4; warps 2..5 take the tile's left half of the
+    // columns and warps 6..9 the right half. Each thread keeps its row's running sums.
     const int quad = warp & 3;
     const int half = (warp - 2) >> 2;
     const uint32_t stg = staging0 + static_cast<uint32_t>(warp - 2) * STAGING_PER_WARP;
+    const bool defer = AR && p.defer_replicas;
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
+    bool pending = false;                 // a region of replica 0 still to copy into the others
+    int pend_row0 = 0, pend_col0 = 0, pend_cols = 0;
     float sum[4][32];
-    for (int tile = pair; ok && tile < num_tiles; tile += pairs) {
-      int mt, nt;
-      raster_by_chunk(tile, tiles_m, p.tiles_n, p.axis, p.chunk_tiles, mt, nt);
-      const int ch = (p.axis == 0 ? mt * TILE_M : nt * BN) / p.chunk;
+    for (int u = pair; ok && u < p.num_units; u += pairs) {
+      int mt, n0;
+      bool wide;
+      ring_pair_unit(p, u, tiles_m, mt, n0, wide);
+      const int ch = (p.axis == 0 ? mt * TILE_M : n0) / p.chunk;
       const int m0 = mt * TILE_M + static_cast<int>(c.rank) * BM;
-      const int n0 = nt * BN;
+      const int cols = wide ? BN / 2 : BN / 4;       // this warp's columns: 128 or 64
+      const int nq = cols / 32;
       for (int j = 0; j < t; ++j) {
         ok = pair_wait_acc_full(c, acc, acc_phase);
         if (!ok) break;
         const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
-                               static_cast<uint32_t>(acc * BN + half * 128);
+                               static_cast<uint32_t>(acc * BN + half * cols);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          uint32_t v[32];
-          tmem_ld32(t_row + q * 32, v);
-          tmem_ld_wait();
-          if (j == 0) {
+          if (q < nq) {
+            uint32_t v[32];
+            tmem_ld32(t_row + q * 32, v);
+            tmem_ld_wait();
+            if (j == 0) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) sum[q][i] = __uint_as_float(v[i]);
-          } else {
+              for (int i = 0; i < 32; ++i) sum[q][i] = __uint_as_float(v[i]);
+            } else {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) sum[q][i] = __fadd_rn(sum[q][i], __uint_as_float(v[i]));
+              for (int i = 0; i < 32; ++i) sum[q][i] = __fadd_rn(sum[q][i], __uint_as_float(v[i]));
+            }
           }
         }
         pair_release_acc(c, acc, lane);
         if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+        if (pending) copy_replica_rows<OUT_BF16>(p, lane, pend_row0, pend_col0, pend_cols, (32 * j) / t, (32 * (j + 1)) / t);
       }
       if (!ok) break;
 #pragma unroll
       for (int q = 0; q < 4; ++q)
-        store_block32<OUT_BF16, AR>(p, stg, lane, sum[q], m0 + quad * 32, n0 + half * 128 + q * 32, ch);
+        if (q < nq) store_block32<OUT_BF16, AR>(p, stg, lane, sum[q], m0 + quad * 32, n0 + half * cols + q * 32, ch, defer);
+      pending = defer;
+      pend_row0 = m0 + quad * 32;
+      pend_col0 = n0 + half * cols;
+      pend_cols = cols;
     }
+    if (ok && pending) copy_replica_rows<OUT_BF16>(p, lane, pend_row0, pend_col0, pend_cols, 0, 32);
   }
   pair_teardown(c, warp, lane, mma_issued, tmem_base);
 }
@@ -1051,6 +1127,14 @@ tp_status launch_ring(RingGemmParams& p, bool pair, cudaStream_t s) {
     const int tiles = ((p.M + 2 * BM - 1) / (2 * BM)) * p.tiles_n;
     int grid = 2 * tiles < sms ? 2 * tiles : (sms & ~1);
     if (grid < 2) grid = 2;
+    // Half-width tiles for a last round that would leave at least half of the pairs idle
+    // (B stored [K][N]: a half tile loads one 64-column box per CTA).
+    const int pairs = grid / 2;
+    const int rem = tiles % pairs;
+    const bool halves = !p.b_km && tiles > pairs && rem > 0 && 2 * rem <= pairs;
+    p.full_units = halves ? tiles - rem : tiles;
+    p.num_units = halves ? tiles + rem : tiles;
+    p.defer_replicas = AR && p.t > 1;
     gemm_ring_pair_kernel<OUT_BF16, AR><<<grid, RING_THREADS, RING_PAIR_SMEM, s>>>(p);
     return check_launch("gemm_ring_pair_kernel");
   }
