@@ -258,7 +258,10 @@ tp_status tp_mlp_fwd_sp(const uint16_t* const* x, int64_t N, int64_t h, int64_t 
  *   case 4 X[B_X, D] . W[D, F_X] (only diagonal blocks as is), fixed by
  *       GATHER_X -> c[i] [B, F/t]; GATHER_W -> c[i] [B/t, F]
  * Partial sums are fp32 and reduced in the ring order above; a bf16 c_dtype rounds once at the end.
- * The workspace (device, >= tp_sharded_matmul_ws_bytes) holds gathered operands or partials. */
+ * The workspace (device, >= tp_sharded_matmul_ws_bytes) holds gathered operands or partials. It is
+ * 0 bytes (ws may be NULL) when the fused row GEMM + ring reduction computes case 2 AllReduce or a
+ * case-3 strategy, i.e. when every reduction chunk is a whole number of 128-row tiles (256-column
+ * tiles for TP_CASE3_RS_F). */
 size_t tp_sharded_matmul_ws_bytes(int case_id, int strategy, int64_t B, int64_t D, int64_t F, int t);
 tp_status tp_sharded_matmul(int case_id, int strategy, const uint16_t* const* x, const uint16_t* const* w,
                             int64_t B, int64_t D, int64_t F, int t, void* const* c, tp_dtype c_dtype,

@@ -242,8 +242,14 @@ size_t tp_sharded_matmul_ws_bytes(int case_id, int strategy, int64_t B, int64_t 
   if (t < 1 || B <= 0 || D <= 0 || F <= 0) return 0;
   const size_t T = static_cast<size_t>(t);
   switch (case_id) {
-    case 2: return strategy == TP_CASE2_ALLGATHER ? T * align256(size_t(B) * D * 2) : T * align256(size_t(B) * F * 4);
-    case 3: return T * align256(size_t(B) * F * 4);
+    case 2:   // AllReduce: no workspace when the fused row GEMM + ring reduction applies
+      if (strategy == TP_CASE2_ALLGATHER) return T * align256(size_t(B) * D * 2);
+      return (B % t == 0 && ring_gemm_fits(B, F, t, 0)) ? 0 : T * align256(size_t(B) * F * 4);
+    case 3: {  // likewise for every case-3 strategy
+      const int axis = strategy == TP_CASE3_RS_F ? 1 : 0;
+      const bool divides = axis == 1 ? F % t == 0 : B % t == 0;
+      return (divides && ring_gemm_fits(B, F, t, axis)) ? 0 : T * align256(size_t(B) * F * 4);
+    }
     case 4: return strategy == TP_CASE4_GATHER_X ? T * align256(size_t(B) * D * 2) : T * align256(size_t(D) * F * 2);
     default: return 0;
   }

@@ -700,8 +700,8 @@ struct RingGemmParams {
   // CTA-pair kernel schedule: units [0, full_units) are 256 x 256 tiles in raster order; the
   // remaining tiles are cut into two 256 x 128 halves each, units [full_units, num_units).
   int full_units, num_units;
-  // AllReduce on CTA pairs: write replica 0 at the tile's end and copy it into the other t - 1
-  // replicas a slice at a time while the next tile's shards run.
+  // AllReduce on CTA pairs with t >= 8: write replica 0 at the tile's end and copy it into the other
+  // t - 1 replicas a slice at a time while the next tile's shards run.
   bool defer_replicas;
   uint32_t* status;
   unsigned long long budget;
@@ -781,22 +781,33 @@ __device__ __forceinline__ void store_block32(const RingGemmParams& p, uint32_t 
 
 // Deferred AllGather leg of the CTA-pair AllReduce: rows [r_begin, r_end) of one warp's region
 // (first row row0, first column col0, ncols columns) are copied from replica 0, which this warp
-// wrote, into replicas 1..t-1. Copying moves bits, so the replicas stay identical.
+// wrote, into replicas 1..t-1. Copying moves bits, so the replicas stay identical. Loads go out in
+// batches of four per lane before their stores, so that a read-back that missed L2 does not
+// serialise the loop.
 template <bool OUT_BF16>
 __device__ __forceinline__ void copy_replica_rows(const RingGemmParams& p, int lane, int row0, int col0, int ncols,
                                                   int r_begin, int r_end) {
   constexpr int PER16 = OUT_BF16 ? 8 : 4;          // elements per 16-byte vector
   constexpr int ESIZE = OUT_BF16 ? 2 : 4;
+  constexpr int BATCH = 4;
   const int vec_per_row = ncols / PER16;
   const int total = (r_end - r_begin) * vec_per_row;
-  for (int idx = lane; idx < total; idx += 32) {
-    const int row = row0 + r_begin + idx / vec_per_row;
-    const int col = col0 + (idx % vec_per_row) * PER16;
-    if (row < p.M && col < p.N) {
-      const int64_t off = (static_cast<int64_t>(row) * p.N + col) * ESIZE;
-      const uint4 v = ld_cg_v4(static_cast<const uint8_t*>(p.out[0]) + off);
-      for (int s = 1; s < p.t; ++s) st_cs_v4(static_cast<uint8_t*>(p.out[s]) + off, v);
+  const uint8_t* src = static_cast<const uint8_t*>(p.out[0]);
+  for (int base = 0; base < total; base += 32 * BATCH) {
+    uint4 v[BATCH];
+    int64_t off[BATCH];
+#pragma unroll
+    for (int b = 0; b < BATCH; ++b) {
+      const int idx = base + 32 * b + lane;
+      const int row = row0 + r_begin + idx / vec_per_row;
+      const int col = col0 + (idx % vec_per_row) * PER16;
+      off[b] = (idx < total && row < p.M && col < p.N) ? (static_cast<int64_t>(row) * p.N + col) * ESIZE : -1;
+      if (off[b] >= 0) v[b] = ld_cg_v4(src + off[b]);
     }
+#pragma unroll
+    for (int b = 0; b < BATCH; ++b)
+      if (off[b] >= 0)
+        for (int s = 1; s < p.t; ++s) st_cs_v4(static_cast<uint8_t*>(p.out[s]) + off[b], v[b]);
   }
 }
 
@@ -934,9 +945,9 @@ __device__ __forceinline__ void ring_pair_unit(const RingGemmParams& p, int u, i
 // gemm_ring_kernel, each CTA summing and storing its own 128 rows of a 256-row pair tile.
 //  * Tiles are 256 x 256. When the last round of tiles would leave at least half of the pairs idle,
 //    those tiles are cut into 256 x 128 halves (MMA N = 128), so that round takes half the time.
-//  * AllReduce: at a tile's end only replica 0 is written; the copies into replicas 1..t-1 are
-//    spread over the next tile's t shard steps (1/t of the rows after each step), so the t-fold
-//    write traffic overlaps the tensor-core work instead of arriving as one burst per tile.
+//  * AllReduce with t >= 8: at a tile's end only replica 0 is written; the copies into replicas
+//    1..t-1 are spread over the next tile's t shard steps (1/t of the rows after each step), so the
+//    t-fold write traffic overlaps the tensor-core work instead of arriving as one burst per tile.
 template <bool OUT_BF16, bool AR>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(RING_THREADS, 1)
     gemm_ring_pair_kernel(const __grid_constant__ RingGemmParams p) {
@@ -1134,7 +1145,9 @@ tp_status launch_ring(RingGemmParams& p, bool pair, cudaStream_t s) {
     const bool halves = !p.b_km && tiles > pairs && rem > 0 && 2 * rem <= pairs;
     p.full_units = halves ? tiles - rem : tiles;
     p.num_units = halves ? tiles + rem : tiles;
-    p.defer_replicas = AR && p.t > 1;
+    // Deferring costs one read-back of the tile and saves a burst of t - 1 copies: measured a gain at
+    // t = 8 (Llama-3-8B down GEMM, 70B layer) and a loss at t = 4 with 0.9 GB replicas (case 3).
+    p.defer_replicas = AR && p.t >= 8;
     gemm_ring_pair_kernel<OUT_BF16, AR><<<grid, RING_THREADS, RING_PAIR_SMEM, s>>>(p);
     return check_launch("gemm_ring_pair_kernel");
   }

@@ -93,8 +93,14 @@ def test_sharded_matmul_workspace_sizes_and_validation():
     B, D, F, t = 8192, 8192, 28672, 4
     assert tp.tp_sharded_matmul_ws_bytes(1, 0, B, D, F, t) == 0
     assert tp.tp_sharded_matmul_ws_bytes(2, tp.TP_CASE2_ALLGATHER, B, D, F, t) == t * B * D * 2
-    assert tp.tp_sharded_matmul_ws_bytes(2, tp.TP_CASE2_ALLREDUCE, B, D, F, t) == t * B * F * 4
-    assert tp.tp_sharded_matmul_ws_bytes(3, tp.TP_CASE3_RS_F, B, D, F, t) == t * B * F * 4
+    # the fused row GEMM + ring reduction needs no workspace when the chunks are whole tiles ...
+    assert tp.tp_sharded_matmul_ws_bytes(2, tp.TP_CASE2_ALLREDUCE, B, D, F, t) == 0
+    assert tp.tp_sharded_matmul_ws_bytes(3, tp.TP_CASE3_RS_F, B, D, F, t) == 0
+    assert tp.tp_sharded_matmul_ws_bytes(3, tp.TP_CASE3_RS_B, B, D, F, t) == 0
+    # ... and the unfused path's fp32 partials otherwise (B/t = 24 rows: no whole 128-row tile)
+    assert tp.tp_sharded_matmul_ws_bytes(2, tp.TP_CASE2_ALLREDUCE, 96, D, F, t) == t * 96 * F * 4
+    assert tp.tp_sharded_matmul_ws_bytes(3, tp.TP_CASE3_RS_B, 96, D, F, t) == t * 96 * F * 4
+    assert tp.tp_sharded_matmul_ws_bytes(3, tp.TP_CASE3_RS_F, B, D, 1000, t) == t * B * 1000 * 4
     assert tp.tp_sharded_matmul_ws_bytes(4, tp.TP_CASE4_GATHER_W, B, D, F, t) == t * D * F * 2
     _expect(tp.TP_ENOSPACE, tp.tp_sharded_matmul, 3, 0, [FAKE] * 4, [FAKE] * 4, 64, 64, 64, 4, [FAKE] * 4, tp.TP_F32,
             FAKE, 10, 0)

@@ -214,6 +214,9 @@ def test_cases_full_size_sampled(case_operands_full, case_id, strategy):
                 shard, rr, cc = (a + b) % t, r, col
             got[a, b] = float(c[shard][rr, cc])
     assert_close(got, ref, GEMM_TOL, f"case {case_id} strategy {strategy}")
+    if layout == "replicated":   # AllReduce: every replica bit-identical at full size
+        for i in range(1, t):
+            assert torch.equal(c[i], c[0]), f"replica {i}"
 
 
 # ---------------------------------------------------------------------------------- 70B-shaped layer
