@@ -384,7 +384,7 @@ def run_gpu(args) -> int:
         gemm_peak = bf16_sust if long_region else bf16_burst
         col_tflops = FLOPS_COL / (avg[0] * 1e-3) / 1e12
         rs_gbs = RS_BYTES / (rs_ms * 1e-3) / 1e9
-        roofline = {"bound": "tensor", "kernel": "gemm_tcgen05_kernel<SwiGLU> (column-parallel gate|up GEMM)",
+        roofline = {"bound": "tensor", "kernel": "gemm_pair_kernel<SwiGLU> (column-parallel gate|up GEMM, CTA pairs)",
                     "achieved": col_tflops, "peak": gemm_peak, "unit": "TFLOP/s", "frac": col_tflops / gemm_peak,
                     "peak_source": f"{src} bf16 {'sustained' if long_region else 'burst'}",
                     "flops_per_launch": FLOPS_COL, "avg_launch_ms": avg[0],
@@ -395,7 +395,7 @@ def run_gpu(args) -> int:
                        "bus_bw_gbs": (T - 1) / T * M_PARTIAL / (rs_ms * 1e-3) / 1e9,
                        "traffic": _traffic("ring_rs_f32_t8", "collectives.cu")}
         row_tflops = FLOPS_ROW / (avg[1] * 1e-3) / 1e12
-        fused_roof = {"bound": "tensor", "kernel": "gemm_ring_kernel<f32,AR> (row GEMM + ring RS + AG)",
+        fused_roof = {"bound": "tensor", "kernel": "gemm_ring_pair_kernel<f32,AR> (row GEMM + ring RS + AG, CTA pairs)",
                       "achieved": row_tflops, "peak": gemm_peak, "unit": "TFLOP/s", "frac": row_tflops / gemm_peak,
                       "flops_per_launch": FLOPS_ROW, "avg_launch_ms": avg[1],
                       "bytes_written_per_launch": T * M_PARTIAL,

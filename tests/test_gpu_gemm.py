@@ -42,6 +42,9 @@ def _run(groups, M, N, K, act, c_dtype, shared_a, seed=0):
     (4, 256, 768, 512, True),     # shared A (column-parallel form)
     (8, 130, 520, 136, False),    # many groups, ragged
     (2, 1024, 1024, 4096, True),  # long K
+    # 80 CTA-pair tiles: more than one round on the 74 pairs of a 148-SM GPU
+    (2, 1024, 2560, 512, False),
+    (2, 1024, 2520, 264, True),   # ... with a ragged N tail and a ragged K
 ])
 def test_gemm_fp32_out(groups, M, N, K, shared):
     got, ref = _run(groups, M, N, K, "none", tp.TP_F32, shared, seed=M + N + K)
@@ -50,7 +53,8 @@ def test_gemm_fp32_out(groups, M, N, K, shared):
 
 
 @pytest.mark.parametrize("act", ["none", "gelu", "gelu_tanh"])
-@pytest.mark.parametrize("groups,M,N,K", [(2, 256, 512, 512), (4, 64, 256, 256), (3, 200, 136, 96)])
+@pytest.mark.parametrize("groups,M,N,K", [(2, 256, 512, 512), (4, 64, 256, 256), (3, 200, 136, 96),
+                                          (2, 1024, 2560, 256)])   # more tiles than CTA pairs
 def test_gemm_bf16_epilogues(act, groups, M, N, K):
     got, ref = _run(groups, M, N, K, act, tp.TP_BF16, shared_a=True, seed=N)
     for g in range(groups):
@@ -59,7 +63,8 @@ def test_gemm_bf16_epilogues(act, groups, M, N, K):
         assert_close(got[g], ref[g], 1e-2, f"{act} group {g} (rounding bound)")
 
 
-@pytest.mark.parametrize("groups,M,N,K", [(1, 128, 128, 64), (2, 256, 384, 512), (8, 192, 136, 264), (8, 512, 1792, 1024)])
+@pytest.mark.parametrize("groups,M,N,K", [(1, 128, 128, 64), (2, 256, 384, 512), (8, 192, 136, 264), (8, 512, 1792, 1024),
+                                          (2, 1024, 1280, 512), (2, 1024, 1224, 264)])   # more tiles than CTA pairs
 def test_gemm_swiglu_pairs_gate_and_up(groups, M, N, K):
     got, ref = _run(groups, M, N, K, "swiglu", tp.TP_BF16, shared_a=True, seed=K)
     for g in range(groups):
