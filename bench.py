@@ -387,6 +387,7 @@ def run_gpu(args) -> int:
         roofline = {"bound": "tensor", "kernel": "gemm_pair_kernel<SwiGLU> (column-parallel gate|up GEMM, CTA pairs)",
                     "achieved": col_tflops, "peak": gemm_peak, "unit": "TFLOP/s", "frac": col_tflops / gemm_peak,
                     "peak_source": f"{src} bf16 {'sustained' if long_region else 'burst'}",
+                    "frac_of_sustained": col_tflops / bf16_sust,
                     "flops_per_launch": FLOPS_COL, "avg_launch_ms": avg[0],
                     "traffic": _traffic("gemm_swiglu_8b", "gemm.cu")}
         roofline_rs = {"bound": "hbm", "kernel": "ring_reduce_kernel<f32,t=8> (standalone ReduceScatter along tokens)",
@@ -397,6 +398,7 @@ def run_gpu(args) -> int:
         row_tflops = FLOPS_ROW / (avg[1] * 1e-3) / 1e12
         fused_roof = {"bound": "tensor", "kernel": "gemm_ring_pair_kernel<f32,AR> (row GEMM + ring RS + AG, CTA pairs)",
                       "achieved": row_tflops, "peak": gemm_peak, "unit": "TFLOP/s", "frac": row_tflops / gemm_peak,
+                      "frac_of_sustained": row_tflops / bf16_sust,
                       "flops_per_launch": FLOPS_ROW, "avg_launch_ms": avg[1],
                       "bytes_written_per_launch": T * M_PARTIAL,
                       "traffic": _traffic("gemm_ring_8b", "gemm.cu")}

@@ -53,6 +53,11 @@ CASES = [
     (8, 2048, 1024, 2600, tp.TP_OUT_RS_AG, 0),  # 88 tiles, N tail: one half tile wholly past N
     (2, 2048, 512, 2560, tp.TP_OUT_RS, 0),
     (4, 1280, 512, 4096, tp.TP_OUT_RS, 1),    # axis 1, 80 tiles
+    # shard-count extremes: t = 1 (a single chunk) and t = 16 (the maximum)
+    (1, 512, 512, 512, tp.TP_OUT_AR, 0),
+    (1, 384, 256, 512, tp.TP_OUT_RS, 1),
+    (16, 4096, 2048, 1024, tp.TP_OUT_RS_AG, 0),   # 256-row chunks: CTA pairs, deferred replica copies
+    (16, 2048, 4096, 512, tp.TP_OUT_RS, 0),       # 128-row chunks: single-CTA kernel
 ]
 
 

@@ -74,6 +74,38 @@ def test_tiny_gelu_mlp_all_modes():
         assert same_bits(rs[r], ar[0][r * N // t:(r + 1) * N // t])
 
 
+# ---------------------------------------------------------------------------------- shard-count extremes
+@pytest.mark.parametrize("N,h,F,t,act", [
+    (512, 256, 1024, 1, "gelu"),        # t = 1: no sharding, the ring is a single chunk
+    (2048, 512, 4096, 16, "swiglu"),    # t = 16 (the maximum): 128-row chunks, single-CTA fused kernel
+    (4096, 512, 4096, 16, "gelu"),      # t = 16: 256-row chunks, CTA pairs, deferred replica copies
+])
+def test_mlp_shard_count_extremes(N, h, F, t, act):
+    d = S.Draw(N + F + t)
+    f = F // t
+    wn = 2 * f if act == "swiglu" else f
+    X = d.normal((N, h), 1.0)
+    w_in = d.normal((t, h, wn), 0.05)
+    w_down = d.normal((t, f, h), 0.05)
+    dX, dw_in, dw_down = cuda(X), cuda(w_in), cuda(w_down)
+    a = tp.TP_ACT_SWIGLU if act == "swiglu" else tp.TP_ACT_GELU
+    res = {mode: _mlp_device(dX, dw_in, dw_down, N, h, F, t, a, mode)
+           for mode in (tp.TP_OUT_PARTIALS, tp.TP_OUT_RS, tp.TP_OUT_AR, tp.TP_OUT_RS_AG)}
+    rows = np.arange(N) if N <= 512 else np.sort(np.random.default_rng(t).choice(N, 32, replace=False))
+    U = OM.mlp_partials(f64(X)[rows], [f64(w) for w in w_in], [f64(w) for w in w_down], act)
+    partials = res[tp.TP_OUT_PARTIALS][1]
+    for r in range(t):
+        assert_close(f64(partials[r])[rows], U[r], GEMM_TOL, f"partial {r}")
+    Y = sum(U)
+    ar = [host_bits(o) for o in res[tp.TP_OUT_AR][2]]
+    rsag = [host_bits(o) for o in res[tp.TP_OUT_RS_AG][2]]
+    rs = [host_bits(o) for o in res[tp.TP_OUT_RS][2]]
+    assert_close(f64(res[tp.TP_OUT_AR][2][0])[rows], Y, GEMM_TOL, "AllReduce")
+    for r in range(t):
+        assert same_bits(ar[r], ar[0]) and same_bits(rsag[r], ar[0]), f"replica {r}"
+        assert same_bits(rs[r], ar[0][r * N // t:(r + 1) * N // t]), f"RS block {r}"
+
+
 # ---------------------------------------------------------------------------------- Llama-3-8B SwiGLU MLP
 @pytest.fixture(scope="module")
 def llama8b():
