@@ -70,10 +70,19 @@ def _traffic(kernel_key: str, source_file: str):
     if not e:
         return None
     src = os.path.join(ROOT, "tensor_sharded_matmul_b200", "csrc", source_file)
-    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    if e.get("source_sha") != sha:
+    if e.get("code_sha") != code_sha(open(src, encoding="utf-8").read()):
         return None
     return e.get("bytes_per_launch")
+
+
+def code_sha(source: str) -> str:
+    """First 16 hex digits of the sha256 of a C++/CUDA source with its comments and blank space
+    removed, so that editing a comment does not retire counters taken from unchanged code."""
+    import re
+    text = re.sub(r"/\*.*?\*/", " ", source, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    text = " ".join(text.split())
+    return hashlib.sha256(text.encode("utf-8")).hexdigest()[:16]
 
 
 class ClockSampler:

@@ -1,35 +1,40 @@
 // bf16 GEMMs on the 5th-generation tensor cores (tcgen05) with fused epilogues.
 //
-// Two persistent, warp-specialised kernels share one TMA -> shared memory -> tcgen05.mma -> TMEM
-// pipeline:
+// Four persistent, warp-specialised kernels share one TMA -> shared memory -> tcgen05.mma -> TMEM
+// pipeline, in a single-CTA form and a CTA-pair form (cluster 2x1, tcgen05 cta_group::2):
 //
-//  gemm_tcgen05_kernel: grouped GEMM C_g = epi(A_g B_g). It serves the column-parallel GEMM
-//    Z_r = act(X W_r), the row-parallel GEMM U_r = Z_r W_r when the partials themselves are wanted
-//    ("张量并行与序列并行", §矩阵乘法的两种切法 and §MLP：先列后行，只通信一次), and the local
-//    products of the sharded-matmul cases ("Scaling Book 入门第 6 章", §6.2). All t shards of one
-//    layer run in ONE launch over the tile space (shard, m-tile, n-tile).
+//  gemm_tcgen05_kernel / gemm_pair_kernel: grouped GEMM C_g = epi(A_g B_g). They serve the
+//    column-parallel GEMM Z_r = act(X W_r), the row-parallel GEMM U_r = Z_r W_r when the partials
+//    themselves are wanted ("张量并行与序列并行", §矩阵乘法的两种切法 and §MLP：先列后行，只通信一次),
+//    and the local products of the sharded-matmul cases ("Scaling Book 入门第 6 章", §6.2). All t
+//    shards of one layer run in ONE launch over the tile space (shard, m-tile, n-tile).
 //
-//  gemm_ring_kernel: the row-parallel GEMM fused with its collective, the one-GPU form of the
-//    pages' collective matmul ("Scaling Book 入门第 6 章", §6.6; "张量并行与序列并行",
-//    §把通信藏到计算后面). For each output tile it computes the t shards' partial tiles
-//    U_s = A_s B_s one after another IN RING ORDER (s = c+1, c+2, ..., c for the tile's chunk c) into
-//    alternating TMEM accumulators. The epilogue adds them into an fp32 running sum in registers, one
-//    binary32 add per shard, which is exactly the ReduceScatter's summation order. It then writes the
-//    tile once: to shard c's output (ReduceScatter) or to all t outputs (AllReduce = ReduceScatter
-//    followed by AllGather), optionally adding a residual and writing a bf16 copy. The fp32 partials
-//    never reach HBM. Each U_s tile comes from the same instruction sequence as
-//    gemm_tcgen05_kernel's, so the results are bit-identical to the unfused GEMM followed by the
-//    ring kernel.
+//  gemm_ring_kernel / gemm_ring_pair_kernel: the row-parallel GEMM fused with its collective, the
+//    one-GPU form of the pages' collective matmul ("Scaling Book 入门第 6 章", §6.6;
+//    "张量并行与序列并行", §把通信藏到计算后面). For each output tile they compute the t shards' partial
+//    tiles U_s = A_s B_s one after another IN RING ORDER (s = c+1, c+2, ..., c for the tile's chunk
+//    c) into alternating TMEM accumulators. The epilogue adds them into an fp32 running sum in
+//    registers, one binary32 add per shard, which is exactly the ReduceScatter's summation order. It
+//    then writes the tile once: to shard c's output (ReduceScatter) or to all t outputs (AllReduce =
+//    ReduceScatter followed by AllGather), optionally adding a residual and writing a bf16 copy. The
+//    fp32 partials never reach HBM. Each U_s tile comes from the same MMA instruction sequence as the
+//    plain GEMM's, so the results are bit-identical to the unfused GEMM followed by the ring kernel.
 //
 // Pipeline (sm_100a):
-//   * warp 0, one lane: TMA producer. A [M,K] is K-major (box 64 x 128, 128-byte swizzle); B [K,N] is
-//     the weight as stored, [in, out] row-major, i.e. MN-major (four 64 x 64 boxes, 128-byte swizzle);
-//   * warp 1, one lane: tcgen05.mma issuer (M=128, N=256, K=16 per instruction, fp32 in TMEM);
-//     4-stage shared-memory ring; two TMEM accumulators of 256 columns, so the epilogue of one unit
-//     overlaps the main loop of the next;
+//   * warp 0, one lane: TMA producer. A [M,K] is K-major (64 x 128 boxes, 128-byte swizzle); B [K,N]
+//     is the weight as stored, [in, out] row-major, i.e. MN-major (64 x 64 boxes, 128-byte swizzle);
+//     the transposed forms (A stored [K][M], B stored [N][K]) swap the box shapes;
+//   * warp 1, one lane: tcgen05.mma issuer, K=16 per instruction, fp32 in TMEM. Single CTA: M=128,
+//     N=256, a 4-stage ring of 48 KB stages. CTA pair: M=256 over the pair (each CTA holds 128 rows
+//     of A and half of B's 256 columns), a 6-stage ring of 32 KB stages per CTA, issued by the
+//     pair's leader, whose barriers count both CTAs' TMA bytes;
+//   * two TMEM accumulators of 256 columns, so the epilogue of one unit overlaps the main loop of the
+//     next;
 //   * the remaining warps: epilogue (tcgen05.ld 32 columns at a time);
 //   * every mbarrier wait is bounded: on expiry the kernel records the site in the status word,
 //     raises a shared abort flag, drains its in-flight copies and MMAs and frees TMEM.
+// No TMA load uses cluster multicast; the pair's commits reach both CTAs through tcgen05.commit's
+// multicast form.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
