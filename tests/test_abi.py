@@ -143,3 +143,16 @@ def test_empty_inputs_are_noops_without_a_gpu():
     _expect(tp.TP_EINVAL, tp.tp_column_linear, 0, -1, 256, 1024, 4, tp.TP_ACT_GELU, 0, 0, 0)
     _expect(tp.TP_EINVAL, tp.tp_grouped_gemm, 1, [FAKE], [FAKE], [FAKE], 64, 64, 0, tp.TP_ACT_NONE, tp.TP_F32, 0)
     _expect(tp.TP_EINVAL, tp.tp_mlp_fwd, 0, 0, 0, 1024, 4, tp.TP_ACT_GELU, 0, 0, 0, None, tp.TP_OUT_RS, [0] * 4, 0)
+
+
+def test_oversized_problems_are_rejected_before_launch():
+    """Sizes past the kernels' 32-bit tile coordinates give TP_ESHAPE on the host (no GPU needed)."""
+    big = 1 << 31
+    _expect(tp.TP_ESHAPE, tp.tp_grouped_gemm, 1, [FAKE], [FAKE], [FAKE], big, 64, 64, tp.TP_ACT_NONE, tp.TP_F32, 0)
+    _expect(tp.TP_ESHAPE, tp.tp_grouped_gemm, 1, [FAKE], [FAKE], [FAKE], 256, 64, big, tp.TP_ACT_NONE, tp.TP_F32, 0)
+    _expect(tp.TP_ESHAPE, tp.tp_grouped_gemm_t, 1, [FAKE], 1, [FAKE], 1, [FAKE], 256, big, 64, tp.TP_F32, 0)
+    _expect(tp.TP_ESHAPE, tp.tp_row_linear_reduce, FAKE, big, 1024, 512, 4, FAKE, tp.TP_OUT_AR, 0, [FAKE] * 4)
+    # the maximum shard count is accepted up to validation, one more is not
+    _expect(tp.TP_EDIVIS, tp.tp_reduce_scatter, [FAKE] * 16, [FAKE] * 16, 24, 16, 0, tp.TP_F32, 16, 0)
+    _expect(tp.TP_EINVAL, tp.tp_mlp_fwd, FAKE, 64, 256, 1024, 17, tp.TP_ACT_GELU, FAKE, FAKE, FAKE, [FAKE] * 17,
+            tp.TP_OUT_PARTIALS, None, 0)
