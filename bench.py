@@ -415,9 +415,9 @@ def run_gpu(args) -> int:
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": n, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": per_step_ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "model": "llama3-8b-mlp", "tokens": N_TOK, "h": H, "F": F, "t": T,
+            "config": {"workload": WORKLOAD, "tokens": N_TOK, "h": H, "F": F, "t": T,
                        "parallelism": f"{T} virtual TP shards per GPU; {n} independent replica(s)",
-                       "l2": "no flush: each step touches ~1.5 GB (weights 336 MiB, partials and outputs 1 GiB) > 126 MB L2"},
+                       "l2": "no flush: each step touches ~1 GB (weights 336 MiB, Z 112 MiB, 8 output replicas 512 MiB) > 126 MB L2"},
             "frac_of_peak_bf16": value / n / gemm_peak,
             "reduce_scatter": {"value": rs_gbs, "unit": "GB/s", "frac_hbm": rs_gbs / hbm},
             "kernels_ms": {"column_gemm_swiglu": avg[0], "row_gemm_rs_ag_fused": avg[1],
