@@ -26,8 +26,9 @@
 //     the transposed forms (A stored [K][M], B stored [N][K]) swap the box shapes;
 //   * warp 1, one lane: tcgen05.mma issuer, K=16 per instruction, fp32 in TMEM. Single CTA: M=128,
 //     N=256, a 4-stage ring of 48 KB stages. CTA pair: M=256 over the pair (each CTA holds 128 rows
-//     of A and half of B's 256 columns), a 6-stage ring of 32 KB stages per CTA, issued by the
-//     pair's leader, whose barriers count both CTAs' TMA bytes;
+//     of A and half of B's 256 columns), a 3-stage ring of 64 KB stages per CTA, each stage two
+//     64-deep k-blocks (eight MMAs per barrier round trip), issued by the pair's leader, whose
+//     barriers count both CTAs' TMA bytes;
 //   * two TMEM accumulators of 256 columns, so the epilogue of one unit overlaps the main loop of the
 //     next;
 //   * the remaining warps: epilogue (tcgen05.ld 32 columns at a time);
@@ -64,9 +65,14 @@ constexpr uint32_t STAGING_PER_WARP = 32 * 128;  // 32 rows x 128 bytes
 constexpr size_t GEMM_SMEM = 1024 + STAGES * (A_STAGE + B_STAGE) + 256;
 // CTA-pair (cta_group::2) variant: a 256 x 256 tile per pair, each CTA holding 128 rows of A and
 // 128 of B's columns per stage, so a 6-stage ring fits.
-constexpr int PAIR_STAGES = 6;
-constexpr uint32_t PAIR_A_STAGE = 128 * BK * 2;  // 16 KiB
-constexpr uint32_t PAIR_B_STAGE = 128 * BK * 2;  // 16 KiB: two 64-wide boxes
+// CTA pairs: a stage holds TWO 64-deep k-blocks (K = 128), so each barrier round trip and each
+// commit covers eight MMAs instead of four. Measured against 6 stages of one k-block: 9-19% faster.
+constexpr int PAIR_KB = 2;                           // k-blocks per stage
+constexpr int PAIR_STAGES = 3;
+constexpr uint32_t PAIR_A_HALF = 128 * BK * 2;       // one k-block of this CTA's 128 A rows: 16 KiB
+constexpr uint32_t PAIR_B_HALF = 128 * BK * 2;       // one k-block of its 128 B columns: 16 KiB
+constexpr uint32_t PAIR_A_STAGE = PAIR_KB * PAIR_A_HALF;   // 32 KiB
+constexpr uint32_t PAIR_B_STAGE = PAIR_KB * PAIR_B_HALF;   // 32 KiB
 constexpr size_t PAIR_SMEM = 1024 + PAIR_STAGES * (PAIR_A_STAGE + PAIR_B_STAGE) + 256;
 constexpr size_t RING_SMEM = 1024 + STAGES * (A_STAGE + B_STAGE) + 8 * STAGING_PER_WARP + 256;
 constexpr size_t RING_PAIR_SMEM = 1024 + PAIR_STAGES * (PAIR_A_STAGE + PAIR_B_STAGE) + 8 * STAGING_PER_WARP + 256;
@@ -500,31 +506,34 @@ __device__ __forceinline__ bool pair_fail(const PairCtl& c, uint32_t site) {
   return false;
 }
 
-// Producer of one CTA: the num_kb k-blocks of one unit. m0 is this CTA's first row, nb its first
-// B column: two 64-wide boxes of `tb` for a full tile, one for a half-width tile (wide == false,
-// B stored [K][N] only).
+// Producer of one CTA: the num_kb k-blocks of one unit, PAIR_KB per stage (a k-block past K loads
+// zeros and is not multiplied). m0 is this CTA's first row, nb its first B column: two 64-wide boxes
+// of `tb` per k-block for a full tile, one for a half-width tile (wide == false, B stored [K][N] only).
 __device__ __forceinline__ bool pair_produce_unit(const PairCtl& c, PairRing& r, const CUtensorMap* ta, int m0,
                                                   const CUtensorMap* tb, int nb, int num_kb, bool wide = true) {
   const uint32_t tx = 2 * (PAIR_A_STAGE + (wide ? PAIR_B_STAGE : PAIR_B_STAGE / 2));
-  for (int kb = 0; kb < num_kb; ++kb) {
+  for (int kb = 0; kb < num_kb; kb += PAIR_KB) {
     if (!mbar_wait_bounded(c.empty0 + 8 * r.stage, r.phase ^ 1u, c.budget, c.abort_flag))
       return pair_fail(c, WAIT_PRODUCER_EMPTY);
     if (c.rank == 0) mbar_arrive_expect_tx(c.full0 + 8 * r.stage, tx);
     const uint32_t fb = c.full0_leader + 8 * r.stage;
-    const uint32_t a_dst = smem_u32(c.sA + r.stage * PAIR_A_STAGE);
-    const uint32_t b_dst = smem_u32(c.sB + r.stage * PAIR_B_STAGE);
-    const int k0 = kb * BK;
-    if (c.a_mn) {                       // A^T [K][M]: two 64(M) x 64(K) boxes of this CTA's 128 rows
-      tma_load_2d_pair(a_dst, ta, m0, k0, fb);
-      tma_load_2d_pair(a_dst + B_BOX, ta, m0 + 64, k0, fb);
-    } else {
-      tma_load_2d_pair(a_dst, ta, k0, m0, fb);
-    }
-    if (c.b_km) {                       // B^T [N][K]: one 64(K) x 128(N) box of this CTA's columns
-      tma_load_2d_pair_hint(b_dst, tb, k0, nb, fb, c.b_policy);
-    } else {
-      tma_load_2d_pair_hint(b_dst, tb, nb, k0, fb, c.b_policy);
-      if (wide) tma_load_2d_pair_hint(b_dst + B_BOX, tb, nb + 64, k0, fb, c.b_policy);
+#pragma unroll
+    for (int h = 0; h < PAIR_KB; ++h) {
+      const uint32_t a_dst = smem_u32(c.sA + r.stage * PAIR_A_STAGE + h * PAIR_A_HALF);
+      const uint32_t b_dst = smem_u32(c.sB + r.stage * PAIR_B_STAGE + h * PAIR_B_HALF);
+      const int k0 = (kb + h) * BK;
+      if (c.a_mn) {                     // A^T [K][M]: two 64(M) x 64(K) boxes of this CTA's 128 rows
+        tma_load_2d_pair(a_dst, ta, m0, k0, fb);
+        tma_load_2d_pair(a_dst + B_BOX, ta, m0 + 64, k0, fb);
+      } else {
+        tma_load_2d_pair(a_dst, ta, k0, m0, fb);
+      }
+      if (c.b_km) {                     // B^T [N][K]: one 64(K) x 128(N) box of this CTA's columns
+        tma_load_2d_pair_hint(b_dst, tb, k0, nb, fb, c.b_policy);
+      } else {
+        tma_load_2d_pair_hint(b_dst, tb, nb, k0, fb, c.b_policy);
+        if (wide) tma_load_2d_pair_hint(b_dst + B_BOX, tb, nb + 64, k0, fb, c.b_policy);
+      }
     }
     r.advance();
   }
@@ -546,21 +555,27 @@ __device__ __forceinline__ bool pair_wait_acc_empty(const PairCtl& c, int acc, u
 }
 
 // Leader's MMA thread: one unit's num_kb k-blocks into d_tmem (M=256 over the pair; N=256, or 128
-// with c.idesc_half).
+// with c.idesc_half), four K=16 MMAs per k-block, one commit per stage. Only k-blocks below num_kb
+// are multiplied, so the MMA sequence is the same as the single-CTA kernels'.
 __device__ __forceinline__ bool pair_mma_unit(const PairCtl& c, PairRing& r, uint32_t d_tmem, int num_kb,
                                               bool& mma_issued, uint32_t idesc) {
-  for (int kb = 0; kb < num_kb; ++kb) {
+  for (int kb = 0; kb < num_kb; kb += PAIR_KB) {
     if (!mbar_wait_bounded(c.full0 + 8 * r.stage, r.phase, c.budget, c.abort_flag)) return pair_fail(c, WAIT_MMA_FULL);
     tc_fence_after();
-    const uint32_t a_base = smem_u32(c.sA + r.stage * PAIR_A_STAGE);
-    const uint32_t b_base = smem_u32(c.sB + r.stage * PAIR_B_STAGE);
 #pragma unroll
-    for (int k = 0; k < BK / 16; ++k) {
-      const uint64_t ad = c.a_mn ? smem_desc_sw128(a_base + 2048u * k, B_BOX, 1024u)
-                                 : smem_desc_sw128(a_base + 32u * k, 16u, 1024u);
-      const uint64_t bd = c.b_km ? smem_desc_sw128(b_base + 32u * k, 16u, 1024u)
-                                 : smem_desc_sw128(b_base + 2048u * k, B_BOX, 1024u);
-      umma_bf16_pair(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+    for (int h = 0; h < PAIR_KB; ++h) {
+      if (kb + h < num_kb) {
+        const uint32_t a_base = smem_u32(c.sA + r.stage * PAIR_A_STAGE + h * PAIR_A_HALF);
+        const uint32_t b_base = smem_u32(c.sB + r.stage * PAIR_B_STAGE + h * PAIR_B_HALF);
+#pragma unroll
+        for (int k = 0; k < BK / 16; ++k) {
+          const uint64_t ad = c.a_mn ? smem_desc_sw128(a_base + 2048u * k, B_BOX, 1024u)
+                                     : smem_desc_sw128(a_base + 32u * k, 16u, 1024u);
+          const uint64_t bd = c.b_km ? smem_desc_sw128(b_base + 32u * k, 16u, 1024u)
+                                     : smem_desc_sw128(b_base + 2048u * k, B_BOX, 1024u);
+          umma_bf16_pair(d_tmem, ad, bd, idesc, (kb + h) != 0 || k != 0 ? 1u : 0u);
+        }
+      }
     }
     mma_issued = true;
     umma_commit_pair_mc(c.empty0 + 8 * r.stage, 0x3);   // frees the stage in both CTAs
