@@ -64,9 +64,9 @@ constexpr int RING_THREADS = 320;                // producer, MMA, 8 epilogue wa
 constexpr uint32_t STAGING_PER_WARP = 32 * 128;  // 32 rows x 128 bytes
 constexpr size_t GEMM_SMEM = 1024 + STAGES * (A_STAGE + B_STAGE) + 256;
 // CTA-pair (cta_group::2) variant: a 256 x 256 tile per pair, each CTA holding 128 rows of A and
-// 128 of B's columns per stage, so a 6-stage ring fits.
-// CTA pairs: a stage holds TWO 64-deep k-blocks (K = 128), so each barrier round trip and each
-// commit covers eight MMAs instead of four. Measured against 6 stages of one k-block: 9-19% faster.
+// 128 of B's columns per k-block. A stage holds TWO 64-deep k-blocks (K = 128), so each barrier
+// round trip and each commit covers eight MMAs instead of four; 3 such stages fit. Measured against
+// 6 stages of one k-block: 9-19% faster (and 2 stages of three k-blocks: 20% slower).
 constexpr int PAIR_KB = 2;                           // k-blocks per stage
 constexpr int PAIR_STAGES = 3;
 constexpr uint32_t PAIR_A_HALF = 128 * BK * 2;       // one k-block of this CTA's 128 A rows: 16 KiB
