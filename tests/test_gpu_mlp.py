@@ -351,3 +351,45 @@ def test_empty_token_count_is_a_noop_then_a_normal_call_matches():
     Y = OM.mlp_unsharded(f64(X), f64(A), f64(B), "gelu")
     for r in range(t):
         assert_close(f64(out[r]), Y, GEMM_TOL, f"replica {r}")
+
+
+# ---------------------------------------------------------------------------------- streams and graphs
+def test_mlp_step_on_a_side_stream_and_in_a_cuda_graph():
+    """The library only enqueues work on the caller's stream: the same MLP step on a side stream, and
+    captured once into a CUDA graph and replayed, gives bit-identical results to the eager call on
+    the default stream (no host synchronisation or allocation on the path)."""
+    N, h, F, t = 1024, 512, 2048, 8
+    d = S.Draw(11)
+    X = cuda(d.normal((N, h), 1.0))
+    w_in = cuda(d.normal((t, h, 2 * F // t), 0.05))
+    w_down = cuda(d.normal((t, F // t, h), 0.05))
+    z = torch.empty((t, N, F // t), dtype=torch.bfloat16, device="cuda")
+
+    def outputs():
+        return [torch.empty((N, h), device="cuda") for _ in range(t)]
+
+    ref = outputs()
+    tp.tp_mlp_fwd(X, N, h, F, t, tp.TP_ACT_SWIGLU, w_in, w_down, z, None, tp.TP_OUT_RS_AG, ref)
+    torch.cuda.synchronize()
+    _status_ok()
+
+    side = torch.cuda.Stream()
+    got_side = outputs()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        tp.tp_mlp_fwd(X, N, h, F, t, tp.TP_ACT_SWIGLU, w_in, w_down, z, None, tp.TP_OUT_RS_AG, got_side, side)
+    side.synchronize()
+
+    got_graph = outputs()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        tp.tp_mlp_fwd(X, N, h, F, t, tp.TP_ACT_SWIGLU, w_in, w_down, z, None, tp.TP_OUT_RS_AG, got_graph)
+    for o in got_graph:
+        o.zero_()
+    g.replay()
+    g.replay()
+    torch.cuda.synchronize()
+    _status_ok()
+    for r in range(t):
+        assert torch.equal(got_side[r], ref[r]), f"side stream, replica {r}"
+        assert torch.equal(got_graph[r], ref[r]), f"graph replay, replica {r}"
