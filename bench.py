@@ -569,6 +569,72 @@ def run_layer70b(args) -> int:
     return 0
 
 
+def run_next(args) -> int:
+    """The rows beyond the forward MLP, on the Llama-3-8B shape (4096 tokens, h=4096, F=14336, t=8):
+    the TP+SP MLP forward (AllGather along tokens fused into the column GEMM's operand loads,
+    ReduceScatter fused into the row GEMM), the MLP's backward pass (dZ, dW_down, activation
+    backward, dW_in, dX with its ring AllReduce), and AllToAll over the 8 fp32 [4096,4096] shard
+    buffers. TFLOP/s counts algorithmic FLOPs (forward 6*N*h*F, backward 12*N*h*F); GB/s counts the
+    bytes a bit copy must move (read t*M, write t*M)."""
+    import torch
+    import synthetic as S
+    import tensor_sharded_matmul_b200 as tp
+    torch.cuda.set_device(0)
+    hbm, burst, sust, _ = _peaks()
+    t, N, h, f = T, N_TOK, H, F // T
+    bf16 = torch.bfloat16
+    X, Wgu, Wd = S.llama8b_mlp(seed=0, device="cuda")
+    w_in = torch.empty((t, h, 2 * f), dtype=bf16, device="cuda")
+    w_down = torch.empty((t, f, h), dtype=bf16, device="cuda")
+    tp.tp_shard_gate_up(Wgu, 2 * F, Wgu.data_ptr() + 2 * F, 2 * F, h, F, t, w_in)
+    tp.tp_shard_rows(Wd, h, F, h, t, w_down)
+    del Wgu, Wd
+    z = torch.empty((t, N, f), dtype=bf16, device="cuda")
+
+    def tensor_line(row, ms, flops):
+        rate = flops / (ms * 1e-3) / 1e12
+        _emit({"config": "next", "row": row, "ms": ms, "tflops": rate, "frac_bf16_peak": rate / burst,
+               "frac_of_sustained": rate / sust, "flops": flops})
+
+    # f1: TP + SP forward
+    x_shards = [X[r * N // t:(r + 1) * N // t].contiguous() for r in range(t)]
+    out_sp = [torch.empty((N // t, h), device="cuda") for _ in range(t)]
+    ms = _time_ms(lambda: tp.tp_mlp_fwd_sp(x_shards, N, h, F, t, tp.TP_ACT_SWIGLU, w_in, w_down, z, out_sp), 50)
+    tensor_line("f1 TP+SP MLP forward (AG fused into the column GEMM, RS fused into the row GEMM)", ms, FLOPS_STEP)
+    del out_sp, x_shards
+
+    # f3: backward, from the forward's own intermediates
+    d = S.Draw(1, "cuda")
+    dY = d.normal((N, h), 1.0)
+    h_pre = torch.empty((t, N, 2 * f), dtype=bf16, device="cuda")
+    tp.tp_column_linear(X, N, h, 2 * F, t, tp.TP_ACT_NONE, w_in, h_pre)
+    tp.tp_column_linear(X, N, h, F, t, tp.TP_ACT_SWIGLU, w_in, z)
+    dz = torch.empty((t, N, f), dtype=bf16, device="cuda")
+    dh = torch.empty((t, N, 2 * f), dtype=bf16, device="cuda")
+    g_in = torch.empty((t, h, 2 * f), device="cuda")
+    g_down = torch.empty((t, f, h), device="cuda")
+    gx = [torch.empty((N, h), device="cuda") for _ in range(t)]
+    ms = _time_ms(lambda: tp.tp_mlp_bwd(X, dY, N, h, F, t, tp.TP_ACT_SWIGLU, w_in, w_down, h_pre, z, dz, dh, g_in,
+                                        g_down, gx), 20)
+    tensor_line("f3 MLP backward (dZ, dW_down, SwiGLU backward, dW_in, dX + ring AllReduce)", ms, 2 * FLOPS_STEP)
+    st, site = tp.tp_device_status(1)
+    if st != tp.TP_OK:
+        print(f"device wait ran out at site {site}", file=sys.stderr)
+        return 3
+    del h_pre, dz, dh, g_in, g_down, gx, dY
+    torch.cuda.empty_cache()
+
+    # f4: AllToAll, split rows / concatenate columns
+    ins = [torch.empty((N, h), device="cuda").normal_() for _ in range(t)]
+    outs = [torch.empty((N // t, t * h), device="cuda") for _ in range(t)]
+    ms = _time_ms(lambda: tp.tp_all_to_all(ins, outs, N, h, 0, 1, tp.TP_F32, t), 50)
+    nbytes = 2 * t * M_PARTIAL
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    _emit({"config": "next", "row": "f4 AllToAll, 8 x fp32 [4096,4096], split rows / concat columns", "ms": ms,
+           "gbs": gbs, "frac_hbm": gbs / hbm, "bytes": nbytes})
+    return 0
+
+
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -576,7 +642,7 @@ def main(argv=None) -> int:
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (profiling runs)")
-    ap.add_argument("--config", choices=["mlp8b", "sweep", "cases", "layer70b"], default="mlp8b",
+    ap.add_argument("--config", choices=["mlp8b", "sweep", "cases", "layer70b", "next"], default="mlp8b",
                     help="mlp8b: the headline step (one JSON line); the others print one line per measurement")
     args = ap.parse_args(argv)
     if args.warmup < 3:
@@ -589,6 +655,8 @@ def main(argv=None) -> int:
         return run_cases(args)
     if args.config == "layer70b":
         return run_layer70b(args)
+    if args.config == "next":
+        return run_next(args)
     return run_gpu(args)
 
 

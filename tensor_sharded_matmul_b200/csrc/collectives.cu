@@ -205,26 +205,44 @@ struct A2AParams {
   int t, split, concat;
 };
 
-template <int ES, int UNIT>
-__global__ void __launch_bounds__(256) all_to_all_kernel(const __grid_constant__ A2AParams p) {
-  constexpr int EPU = UNIT / ES;
-  const int64_t per_out = p.orow * p.ocol / EPU;
-  const int64_t units = per_out * p.t;
-  for (int64_t u = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; u < units;
-       u += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int j = static_cast<int>(u / per_out);
-    const int64_t e = (u - j * per_out) * EPU;
-    const int64_t r = e / p.ocol, col = e - r * p.ocol;
-    const int i = static_cast<int>(p.concat == 0 ? r / p.pr : col / p.pc);      // source shard
-    const int64_t lr = p.concat == 0 ? r - i * p.pr : r;
-    const int64_t lc = p.concat == 0 ? col : col - i * p.pc;
-    const int64_t sr = p.split == 0 ? j * p.pr + lr : lr;
-    const int64_t sc = p.split == 0 ? lc : j * p.pc + lc;
+// One task = one contiguous run of a piece: destination shard j, source shard i, row lr of the
+// piece. The run is pc elements long on both sides, so a block copies it with plain coalesced
+// vectors and all index arithmetic happens once per run. Loads go out four per thread before their
+// stores.
+template <int ES, bool VEC>
+__global__ void __launch_bounds__(256, 4) all_to_all_kernel(const __grid_constant__ A2AParams p) {
+  const int64_t P = p.pr;                                  // rows per piece
+  const int64_t L = p.pc;                                  // elements per run
+  const int64_t per_j = static_cast<int64_t>(p.t) * P;
+  const int64_t tasks = static_cast<int64_t>(p.t) * per_j;
+  for (int64_t task = blockIdx.x; task < tasks; task += gridDim.x) {
+    const int j = static_cast<int>(task / per_j);
+    const int64_t rem = task - j * per_j;
+    const int i = static_cast<int>(rem / P);
+    const int64_t lr = rem - i * P;
+    const int64_t sr = p.split == 0 ? j * P + lr : lr;     // source row and first column
+    const int64_t sc = p.split == 0 ? 0 : j * L;
+    const int64_t dr = p.concat == 0 ? i * P + lr : lr;    // destination row and first column
+    const int64_t dc = p.concat == 0 ? 0 : i * L;
     const char* src = static_cast<const char*>(p.in[i]) + (sr * p.cols + sc) * ES;
-    char* dst = static_cast<char*>(p.out[j]) + e * ES;
-    if constexpr (UNIT == 16) st_v4(dst, ld_nc_v4(src));
-    else if constexpr (ES == 4) *reinterpret_cast<uint32_t*>(dst) = *reinterpret_cast<const uint32_t*>(src);
-    else *reinterpret_cast<uint16_t*>(dst) = *reinterpret_cast<const uint16_t*>(src);
+    char* dst = static_cast<char*>(p.out[j]) + (dr * p.ocol + dc) * ES;
+    if constexpr (VEC) {
+      const int64_t nv = L * ES / 16;
+      for (int64_t v = threadIdx.x; v < nv; v += 4 * static_cast<int64_t>(blockDim.x)) {
+        uint4 x[4];
+#pragma unroll
+        for (int b = 0; b < 4; ++b)
+          if (v + b * blockDim.x < nv) x[b] = ld_nc_v4(src + (v + b * blockDim.x) * 16);
+#pragma unroll
+        for (int b = 0; b < 4; ++b)
+          if (v + b * blockDim.x < nv) st_v4(dst + (v + b * blockDim.x) * 16, x[b]);
+      }
+    } else {
+      for (int64_t e = threadIdx.x; e < L; e += blockDim.x) {
+        if constexpr (ES == 4) reinterpret_cast<uint32_t*>(dst)[e] = reinterpret_cast<const uint32_t*>(src)[e];
+        else reinterpret_cast<uint16_t*>(dst)[e] = reinterpret_cast<const uint16_t*>(src)[e];
+      }
+    }
   }
 }
 
@@ -353,14 +371,16 @@ tp_status all_to_all(const void* const* in, void* const* out, int64_t rows, int6
   // a vector never straddles a piece: the piece width, both row lengths and every column offset
   // are multiples of the vector length
   const bool vec = all16 && p.pc % epu == 0 && cols % epu == 0 && p.ocol % epu == 0;
-  const int64_t units = t * p.orow * p.ocol / (vec ? epu : 1);
-  const int blocks = grid_for(units);
+  const int64_t tasks = static_cast<int64_t>(t) * t * p.pr;     // one block-sized copy per run
+  const int cap = sm_count() * 4;                               // 4 resident blocks per SM
+  if (cap <= 0) return fail(TP_ECUDA, "cannot query the SM count");
+  const int blocks = static_cast<int>(tasks < cap ? tasks : cap);
   if (es == 4) {
-    if (vec) all_to_all_kernel<4, 16><<<blocks, 256, 0, stream>>>(p);
-    else all_to_all_kernel<4, 4><<<blocks, 256, 0, stream>>>(p);
+    if (vec) all_to_all_kernel<4, true><<<blocks, 256, 0, stream>>>(p);
+    else all_to_all_kernel<4, false><<<blocks, 256, 0, stream>>>(p);
   } else {
-    if (vec) all_to_all_kernel<2, 16><<<blocks, 256, 0, stream>>>(p);
-    else all_to_all_kernel<2, 2><<<blocks, 256, 0, stream>>>(p);
+    if (vec) all_to_all_kernel<2, true><<<blocks, 256, 0, stream>>>(p);
+    else all_to_all_kernel<2, false><<<blocks, 256, 0, stream>>>(p);
   }
   return check_launch("all_to_all_kernel");
 }
