@@ -58,6 +58,9 @@ CASES = [
     (1, 384, 256, 512, tp.TP_OUT_RS, 1),
     (16, 4096, 2048, 1024, tp.TP_OUT_RS_AG, 0),   # 256-row chunks: CTA pairs, deferred replica copies
     (16, 2048, 4096, 512, tp.TP_OUT_RS, 0),       # 128-row chunks: single-CTA kernel
+    # odd k-block counts per shard on CTA pairs (two k-blocks per pipeline stage)
+    (4, 1024, 768, 512, tp.TP_OUT_AR, 0),         # 192 per shard: three k-blocks
+    (2, 512, 80, 512, tp.TP_OUT_RS, 0),           # 40 per shard: one ragged k-block
 ]
 
 

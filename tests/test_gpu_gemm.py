@@ -45,6 +45,9 @@ def _run(groups, M, N, K, act, c_dtype, shared_a, seed=0):
     # 80 CTA-pair tiles: more than one round on the 74 pairs of a 148-SM GPU
     (2, 1024, 2560, 512, False),
     (2, 1024, 2520, 264, True),   # ... with a ragged N tail and a ragged K
+    # CTA pairs take two k-blocks per pipeline stage: odd k-block counts leave the last stage half used
+    (2, 256, 256, 64, False),     # one k-block
+    (1, 512, 512, 136, True),     # three k-blocks, the last ragged
 ])
 def test_gemm_fp32_out(groups, M, N, K, shared):
     got, ref = _run(groups, M, N, K, "none", tp.TP_F32, shared, seed=M + N + K)
