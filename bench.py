@@ -380,6 +380,17 @@ def run_gpu(args) -> int:
     torch.cuda.synchronize()
     e2e_ms = e_start.elapsed_time(e_stop)
 
+    # the copy-out alone (one 64 MiB replica to pinned host memory), for the e2e bound
+    d_start, d_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    d_iters = 10
+    with torch.cuda.stream(s_out):
+        d_start.record(s_out)
+        for _ in range(d_iters):
+            y_host[0].copy_(outs[0][0], non_blocking=True)
+        d_stop.record(s_out)
+    torch.cuda.synchronize()
+    d2h_gbs = d_iters * N_TOK * H * 4 / (d_start.elapsed_time(d_stop) * 1e-3) / 1e9
+
     # ---- max over ranks ------------------------------------------------------------------------
     total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dist, dev)
     n = ws
@@ -427,6 +438,7 @@ def run_gpu(args) -> int:
             "roofline": roofline, "roofline_fused_row_reduce": fused_roof, "roofline_reduce_scatter": roofline_rs,
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": X.numel() * 2,
                     "d2h_bytes_per_step": N_TOK * H * 4, "ms_per_step": e2e_ms / args.steps,
+                    "d2h_alone_gbs": d2h_gbs,
                     "how": "tp_mlp_fwd per step; pinned H2D of X and D2H of one reduced replica on separate "
                            "streams, double-buffered, overlapping the neighbouring steps"},
             "gpu_launches": 2 * args.steps,
