@@ -10,6 +10,7 @@
 //   ReduceScatter: reads t*M bytes, writes M.
 //   AllReduce: reads t*M, writes t*M.
 //   AllGather: reads M, writes t*M.
+//   AllToAll (a bit copy, [CH05] §5.3): reads t*M, writes t*M.
 // No atomics, no reassociation, and the result does not depend on grid size.
 // Memory traffic is coalesced 16-byte vectors; grids are a multiple of the SM count with
 // grid-stride loops. bf16 inputs are widened (exact), summed in binary32 and rounded once to bf16
@@ -195,7 +196,8 @@ __global__ void __launch_bounds__(256) ring_gather_kernel(const __grid_constant_
 }
 
 // AllToAll: out[j] = concatenation along concat_axis of piece j (split along split_axis) of every
-// shard's buffer. Each output element has exactly one source; UNIT bytes are moved per step.
+// shard's buffer. Each output element has exactly one source, and each row of a piece lands as one
+// contiguous run of an output row.
 struct A2AParams {
   const void* in[TP_MAX_SHARDS];
   void* out[TP_MAX_SHARDS];
