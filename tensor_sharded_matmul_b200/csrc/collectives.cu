@@ -10,7 +10,7 @@
 //   ReduceScatter: reads t*M bytes, writes M.
 //   AllReduce: reads t*M, writes t*M.
 //   AllGather: reads M, writes t*M.
-//   AllToAll (a bit copy, [CH05] §5.3): reads t*M, writes t*M.
+//   AllToAll (a bit copy, "Scaling Book 入门第 5 章", §5.3): reads t*M, writes t*M.
 // No atomics, no reassociation, and the result does not depend on grid size.
 // Memory traffic is coalesced 16-byte vectors; grids are a multiple of the SM count with
 // grid-stride loops. bf16 inputs are widened (exact), summed in binary32 and rounded once to bf16
