@@ -49,7 +49,7 @@ typedef enum {
   TP_EALIGN = 4,        /* pointer or row stride not 16-byte aligned */
   TP_ECUDA = 5,         /* a CUDA runtime/driver call failed */
   TP_ETIMEOUT = 6,      /* a bounded device-side wait ran out (reported by tp_device_status) */
-  TP_EUNSUPPORTED = 7,  /* valid request this build does not implement */
+  TP_EUNSUPPORTED = 7,  /* valid request the library does not implement */
   TP_ENOSPACE = 8       /* a caller-supplied workspace is too small */
 } tp_status;
 

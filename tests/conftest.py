@@ -18,8 +18,8 @@ def pytest_configure(config):
 
 
 def pytest_collection_modifyitems(config, items):
-    # A GPU test on a machine without a GPU is a configuration error on the GPU machine, but on the
-    # CPU box the driver selects -m "not gpu"; skip (do not fail) when no device is visible.
+    # GPU tests need a CUDA device; on a host without one they are skipped (CPU runs select
+    # -m "not gpu" anyway), so that a plain `pytest tests` still works there.
     import torch
     if torch.cuda.is_available():
         return
