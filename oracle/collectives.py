@@ -17,6 +17,10 @@ Reading of what the pages leave open (the pages never state a summation order):
     therefore summed as (((U[c+1] + U[c+2]) + U[c+3]) + ... ) + U[c] (indices mod t), left to right.
   * fp32 payloads are accumulated in binary32 (one IEEE rounding per add). bf16 payloads are widened
     to binary32, accumulated in the same order and rounded once to bf16 at the end.
+  * Optional per-hop rounding for bf16 (rounding="hop"): read literally, each device of the ring holds
+    and passes on its running partial in the payload's own type, so when the links carry bf16 the
+    partial is rounded to bf16 after every add (binary32 add, then round to nearest-even bf16), as
+    a ring whose buffers are bf16 does. The default ("end") keeps the partial in binary32.
   * Chunk r of a [rows, cols] buffer is the row block [r*rows/t, (r+1)*rows/t) for axis 0 and the
     column block [r*cols/t, (r+1)*cols/t) for axis 1; AllGather concatenates in shard order.
   * In the bidirectional AllGather with even N, the antipodal shard arrives at the last step through
@@ -81,15 +85,24 @@ def _from_f32(x: np.ndarray, dtype: str) -> np.ndarray:
     return f32_to_bf16_bits(x) if dtype == "bf16" else np.asarray(x, dtype=np.float32)
 
 
-def reduce_scatter(bufs, axis: int = 0, dtype: str = "f32", out_dtype: str | None = None):
+def _bf16_hop_add(a, b):
+    """One hop of a ring whose links carry bf16: binary32 add, then the partial rounded to bf16."""
+    return bf16_bits_to_f32(f32_to_bf16_bits(np.add(a, b, dtype=np.float32)))
+
+
+def reduce_scatter(bufs, axis: int = 0, dtype: str = "f32", out_dtype: str | None = None, rounding: str = "end"):
     """Ring ReduceScatter of t full-size buffers (2-D numpy arrays: float32, or uint16 bf16 bits).
 
     Returns t arrays, the reduced chunk r for shard r, in ``out_dtype`` (default = ``dtype``).
-    Accumulation is binary32 in the ring order described in the module docstring."""
+    Accumulation is binary32 in the ring order described in the module docstring; with
+    ``rounding="hop"`` (bf16 only) the running partial is rounded to bf16 after every add."""
     out_dtype = out_dtype or dtype
+    if rounding not in ("end", "hop") or (rounding == "hop" and (dtype, out_dtype) != ("bf16", "bf16")):
+        raise ValueError("per-hop rounding is a bf16 -> bf16 mode")
     t = len(bufs)
     own = [_split(_as_f32(b, dtype), t, axis) for b in bufs]
-    held = ring_reduce_scatter_steps(own, lambda a, b: np.add(a, b, dtype=np.float32))
+    add = _bf16_hop_add if rounding == "hop" else (lambda a, b: np.add(a, b, dtype=np.float32))
+    held = ring_reduce_scatter_steps(own, add)
     return [_from_f32(h.copy(), out_dtype) for h in held]
 
 
@@ -159,10 +172,11 @@ def all_gather(bufs, axis: int = 0):
     return [np.concatenate([hold[i][k] for k in range(t)], axis=axis) for i in range(t)]
 
 
-def all_reduce(bufs, dtype: str = "f32", out_dtype: str | None = None):
+def all_reduce(bufs, dtype: str = "f32", out_dtype: str | None = None, rounding: str = "end"):
     """AllReduce = ReduceScatter (along rows) followed by AllGather: every shard ends with the full
-    ring-ordered sum. With bf16 the one rounding happens at the end of the ReduceScatter."""
-    rs = reduce_scatter(bufs, axis=0, dtype=dtype, out_dtype=out_dtype)
+    ring-ordered sum. With bf16 the one rounding happens at the end of the ReduceScatter (or after
+    every hop, with rounding="hop")."""
+    rs = reduce_scatter(bufs, axis=0, dtype=dtype, out_dtype=out_dtype, rounding=rounding)
     return all_gather(rs, axis=0)
 
 

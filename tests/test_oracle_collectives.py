@@ -228,3 +228,45 @@ def test_every_chunk_gets_every_shard_exactly_once(t):
     for c, order in enumerate(prov):
         assert sorted(order) == list(range(t)) and order[-1] == c
     assert list(itertools.chain.from_iterable(prov)).count(0) == t
+
+
+# ------------------------------------------------------------------------------------ per-hop bf16 mode
+def test_per_hop_bf16_hand_example():
+    # t = 3, chunk 0 is summed in the ring order U[1], U[2], U[0]. With U[1] = 1 and U[2] = U[0] = 2^-8:
+    #   rounding once at the end: 1 + 2^-8 + 2^-8 = 1 + 2^-7, exactly a bf16 value (0x3F81);
+    #   rounding after every hop: 1 + 2^-8 is a tie between 1 and 1 + 2^-7 and goes to the even 1
+    #   (0x3F80), and so does the second hop.
+    one, small = 0x3F80, 0x3B80          # bf16 bits of 1.0 and 2^-8
+    assert float(bf16_bits_to_f32(np.uint16(small))) == 2.0 ** -8
+    bufs = [np.array([[v], [0], [0]], dtype=np.uint16) for v in (small, one, small)]
+    end = C.reduce_scatter(bufs, axis=0, dtype="bf16")
+    hop = C.reduce_scatter(bufs, axis=0, dtype="bf16", rounding="hop")
+    assert int(end[0][0, 0]) == 0x3F81
+    assert int(hop[0][0, 0]) == 0x3F80
+
+
+@pytest.mark.parametrize("t", [2, 3, 4, 8])
+def test_per_hop_bf16_equals_sequential_bf16_adds(t):
+    # A ring whose links carry bf16 adds one bf16 value at a time and keeps a bf16 partial: exactly
+    # torch's bf16 tensor addition (binary32 add, round to nearest-even) applied in the ring order.
+    g = torch.Generator().manual_seed(40 + t)
+    xs = [torch.randn(t * 16, 24, generator=g).mul(torch.exp(torch.randn(1, generator=g))).to(torch.bfloat16)
+          for _ in range(t)]
+    bits = [x.view(torch.int16).numpy().view(np.uint16) for x in xs]
+    hop = C.reduce_scatter(bits, axis=0, dtype="bf16", rounding="hop")
+    rows = 16
+    for c in range(t):
+        acc = xs[(c + 1) % t][c * rows:(c + 1) * rows]
+        for k in range(2, t + 1):
+            acc = acc + xs[(c + k) % t][c * rows:(c + 1) * rows]
+        ref = acc.view(torch.int16).numpy().view(np.uint16)
+        assert np.array_equal(hop[c], ref), c
+    # and the default mode differs somewhere on this data (a single rounding at the end)
+    if t >= 3:
+        end = C.reduce_scatter(bits, axis=0, dtype="bf16")
+        assert any(not np.array_equal(a, b) for a, b in zip(hop, end))
+
+
+def test_per_hop_mode_is_bf16_only():
+    with pytest.raises(ValueError):
+        C.reduce_scatter([np.zeros((2, 2), np.float32)] * 2, dtype="f32", rounding="hop")
