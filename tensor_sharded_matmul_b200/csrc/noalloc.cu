@@ -68,19 +68,36 @@ extern "C" tp_status tp_mlp_fwd_noalloc(const uint16_t* x, int64_t N, int64_t h,
   if (N < 0 || h <= 0 || F <= 0) return fail(TP_EINVAL, "negative size or empty hidden/F dimension");
   if (N == 0) return TP_OK;                              // no tokens: nothing to compute
   if (mode < TP_OUT_PARTIALS || mode > TP_OUT_RS_AG) return fail(TP_EINVAL, "bad reduce mode");
-  // Scratch: Z as bf16 [t][N][F/t], plus t fp32 [N, h] partials unless the caller's outputs hold them.
-  const size_t z_bytes = round256(size_t(N) * size_t(F) * 2);
-  const size_t part_bytes = round256(size_t(N) * size_t(h) * 4);
-  const size_t need = z_bytes + (mode == TP_OUT_PARTIALS ? 0 : size_t(t) * part_bytes);
-  if (need > TP_MLP_NOALLOC_SCRATCH_BYTES)
-    return fail(TP_ENOSPACE, "this request needs %zu bytes of scratch; the built-in array holds %u",
-                need, (unsigned)TP_MLP_NOALLOC_SCRATCH_BYTES);
+  // Scratch: Z as bf16 [t][N][F/t], plus t fp32 [N, h] partials when a reducing mode takes the
+  // unfused path. When (N/t) % 128 == 0 the row GEMM is fused with its reduction and never touches
+  // partials. Every size is bounded before it is multiplied, so no product can wrap around.
+  const uint64_t cap = TP_MLP_NOALLOC_SCRATCH_BYTES;
+  const uint64_t n = static_cast<uint64_t>(N);
+  if (static_cast<uint64_t>(F) > cap / 2 || n > cap / (2 * static_cast<uint64_t>(F)))
+    return fail(TP_ENOSPACE, "the activations need more scratch than the built-in %u-byte array holds",
+                (unsigned)TP_MLP_NOALLOC_SCRATCH_BYTES);
+  const size_t z_bytes = round256(n * static_cast<uint64_t>(F) * 2);
+  const bool fused = mode != TP_OUT_PARTIALS && ring_gemm_fits(N, h, t, 0);
+  const bool use_partials = mode != TP_OUT_PARTIALS && !fused;
+  size_t part_bytes = 0;
+  if (use_partials) {
+    if (static_cast<uint64_t>(h) > cap / 4 || n > cap / (4 * static_cast<uint64_t>(h)))
+      return fail(TP_ENOSPACE, "the partial sums need more scratch than the built-in %u-byte array holds",
+                  (unsigned)TP_MLP_NOALLOC_SCRATCH_BYTES);
+    part_bytes = round256(n * static_cast<uint64_t>(h) * 4);
+  }
+  const uint64_t need = z_bytes + static_cast<uint64_t>(t) * part_bytes;   // t <= 16: no wrap
+  if (need > cap)
+    return fail(TP_ENOSPACE, "this request needs %llu bytes of scratch; the built-in array holds %u",
+                (unsigned long long)need, (unsigned)TP_MLP_NOALLOC_SCRATCH_BYTES);
   tp_status st = TP_OK;
   char* base = static_cast<char*>(scratch_address(&st));
   if (base == nullptr) return st;
   uint16_t* z = reinterpret_cast<uint16_t*>(base);
   if (mode == TP_OUT_PARTIALS)   // the partials are the result: write them straight into out
     return tp_mlp_fwd(x, N, h, F, t, act, w_in, w_down, z, out, mode, nullptr, stream);
+  if (!use_partials)             // the fused row GEMM + reduction keeps the partials on chip
+    return tp_mlp_fwd(x, N, h, F, t, act, w_in, w_down, z, nullptr, mode, out, stream);
   float* partials[TP_MAX_SHARDS];
   for (int r = 0; r < t; ++r) partials[r] = reinterpret_cast<float*>(base + z_bytes + size_t(r) * part_bytes);
   return tp_mlp_fwd(x, N, h, F, t, act, w_in, w_down, z, partials, mode, out, stream);

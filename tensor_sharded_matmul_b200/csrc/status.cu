@@ -89,7 +89,7 @@ const char* tp_status_str(tp_status s) {
     case TP_ECUDA: return "CUDA error";
     case TP_ETIMEOUT: return "a bounded device wait ran out";
     case TP_EUNSUPPORTED: return "unsupported";
-    case TP_ENOSPACE: return "workspace too small";
+    case TP_ENOSPACE: return "workspace too small (the caller's, or the built-in no-alloc array)";
   }
   return "unknown status";
 }

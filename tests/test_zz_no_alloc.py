@@ -7,16 +7,18 @@ synchronise the device. For them the library keeps the MLP's scratch (activation
 sums) in a fixed array of its own.
 
 This test calls that entry point through the C ABI twice in a row, on different shapes, inputs and
-modes. It compares each result with tp_mlp_fwd's on the same inputs, within the tolerance the other
-GEMM-derived outputs use. It also checks that a request too large for the array is refused. It does
-not depend on other tests having run first.
+modes. Both entry points launch the same kernels on the same inputs, so each result must equal
+tp_mlp_fwd's bit for bit; a tolerance could hide stale scratch or a wrong offset inside the array.
+Shapes with (N/t) % 128 == 0 take the fused row GEMM + reduction, which needs no room for the fp32
+partials, so the Llama-3-8B-shaped MLP on 1024 tokens (29.4 MB of activations) fits the array. It
+also checks that a request too large for the array is refused. It does not depend on other tests
+having run first.
 """
 import pytest
 import torch
 
 import synthetic as S
 import tensor_sharded_matmul_b200 as tp
-from gpu_util import GEMM_TOL, assert_close, f64
 
 pytestmark = pytest.mark.gpu
 
@@ -53,7 +55,7 @@ def _check(N, h, F, t, act, mode, seed):
     st, site = tp.tp_device_status(1)
     assert st == tp.TP_OK, f"device wait site {site}"
     for r in range(t):
-        assert_close(f64(got[r]), f64(ref[r]), GEMM_TOL, f"shard {r}")
+        assert torch.equal(got[r], ref[r]), f"shard {r} differs from tp_mlp_fwd"
 
 
 def test_two_calls_in_a_row_match_tp_mlp_fwd():
@@ -67,6 +69,14 @@ def test_two_calls_in_a_row_match_tp_mlp_fwd():
 def test_partials_and_reduce_scatter_modes():
     _check(N=128, h=512, F=2048, t=8, act=tp.TP_ACT_SWIGLU, mode=tp.TP_OUT_PARTIALS, seed=3)
     _check(N=128, h=512, F=2048, t=8, act=tp.TP_ACT_SWIGLU, mode=tp.TP_OUT_RS, seed=4)
+
+
+def test_fused_path_fits_where_partials_would_not():
+    # N/t = 128: the row GEMM is fused with its AllReduce, so only Z (1024 x 14336 bf16, 29.4 MB) needs
+    # the array; the unfused path's 8 fp32 [1024, 4096] partials (134 MB) would not fit.
+    _check(N=1024, h=4096, F=14336, t=8, act=tp.TP_ACT_SWIGLU, mode=tp.TP_OUT_RS_AG, seed=5)
+    # and a small fused ReduceScatter right after it, on the array the first call left filled
+    _check(N=1024, h=512, F=2048, t=8, act=tp.TP_ACT_GELU, mode=tp.TP_OUT_RS, seed=6)
 
 
 def test_request_beyond_the_array_is_refused():
