@@ -50,10 +50,15 @@ typedef enum {
   TP_ECUDA = 5,         /* a CUDA runtime/driver call failed */
   TP_ETIMEOUT = 6,      /* a bounded device-side wait ran out (reported by tp_device_status) */
   TP_EUNSUPPORTED = 7,  /* valid request the library does not implement */
-  TP_ENOSPACE = 8       /* a caller-supplied workspace is too small */
+  TP_ENOSPACE = 8       /* a workspace is too small: the caller's, or the built-in array of
+                           tp_mlp_fwd_noalloc */
 } tp_status;
 
-typedef enum { TP_F32 = 0, TP_BF16 = 1 } tp_dtype;
+/* Element types. TP_BF16_RING is bf16 storage for the ring collectives only (tp_reduce_scatter,
+ * tp_all_reduce, tp_all_gather): the running partial is rounded to bf16 after every add, as a ring
+ * whose links carry bf16 does. The default bf16 mode (TP_BF16) keeps the partial in binary32 and
+ * rounds once at the end. */
+typedef enum { TP_F32 = 0, TP_BF16 = 1, TP_BF16_RING = 2 } tp_dtype;
 
 /* Activation applied in the column-parallel GEMM's epilogue. It is element-wise, so each shard
  * applies it to its own columns ([TPSP] §MLP：先列后行，只通信一次). GELU is the exact erf form.
@@ -127,7 +132,9 @@ tp_status tp_shard_qkv(const uint16_t* w_q, int64_t ld_q, const uint16_t* w_k, i
  * Summation order (the pages fix the ring, device i passing to i+1 and accumulating at every step,
  * and that device r ends with chunk r; the order of the adds follows from that): chunk c is
  * (((U[c+1] + U[c+2]) + U[c+3]) + ... ) + U[c], indices mod t, one binary32 add at a time. bf16 inputs
- * are widened to binary32, summed in that order and rounded once to bf16 (nearest-even).
+ * are widened to binary32, summed in that order and rounded once to bf16 (nearest-even). With
+ * TP_BF16_RING (optional, NCCL-like) every add is followed by a rounding to bf16 instead: the partial
+ * a device passes on ([CH05] §5.2, §5.3) is held in the payload's type.
  * Chunk r is the row block [r*rows/t, (r+1)*rows/t) (axis 0) or column block (axis 1).
  * Results are bit-exact and independent of launch shape; no atomics are used.
  * ------------------------------------------------------------------------------------------------ */
@@ -259,9 +266,14 @@ tp_status tp_mlp_fwd_sp(const uint16_t* const* x, int64_t N, int64_t h, int64_t 
  *       GATHER_X -> c[i] [B, F/t]; GATHER_W -> c[i] [B/t, F]
  * Partial sums are fp32 and reduced in the ring order above; a bf16 c_dtype rounds once at the end.
  * The workspace (device, >= tp_sharded_matmul_ws_bytes) holds gathered operands or partials. It is
- * 0 bytes (ws may be NULL) when the fused row GEMM + ring reduction computes case 2 AllReduce or a
- * case-3 strategy, i.e. when every reduction chunk is a whole number of 128-row tiles (256-column
- * tiles for TP_CASE3_RS_F). */
+ * 0 bytes (ws may be NULL)
+ *   - when the fused row GEMM + ring reduction computes case 2 AllReduce or a case-3 strategy, i.e.
+ *     when every reduction chunk is a whole number of 128-row tiles (256-column tiles for RS_F);
+ *   - when the GEMM reads the gathered operand's pieces where they lie instead of a gathered copy
+ *     ([CH06] §6.6, the gather folded into the matmul): case 2 AllGather with (D/t) % 64 == 0
+ *     (each k-block of X read from the shard that holds it), case 4 GATHER_X with (B/t) % 128 == 0
+ *     (each 128-row tile of X likewise), case 4 GATHER_W with (F/t) % 64 == 0 (each 64-column box
+ *     of W likewise). Otherwise the gather is materialised in the workspace, one copy per shard. */
 size_t tp_sharded_matmul_ws_bytes(int case_id, int strategy, int64_t B, int64_t D, int64_t F, int t);
 tp_status tp_sharded_matmul(int case_id, int strategy, const uint16_t* const* x, const uint16_t* const* w,
                             int64_t B, int64_t D, int64_t F, int t, void* const* c, tp_dtype c_dtype,
@@ -295,8 +307,11 @@ tp_status tp_layer_fwd(const uint16_t* x, const uint16_t* const* o, int64_t N, i
  * Same computation, arguments and results as tp_mlp_fwd, minus z_ws and partials. The activations
  * and the fp32 partials live in one array of TP_MLP_NOALLOC_SCRATCH_BYTES compiled into the library,
  * which every GPU that loads the library holds until the process exits.
- *   - Requests needing more than that (N*F*2 bytes, plus t*N*h*4 unless mode is TP_OUT_PARTIALS, each
- *     rounded up to 256) return TP_ENOSPACE before any launch.
+ *   - The scratch needed is N*F*2 bytes (Z), rounded up to 256, plus t*N*h*4 (the fp32 partials,
+ *     each rounded up to 256) only when a reducing mode takes the unfused path, i.e. when
+ *     (N/t) % 128 != 0; with (N/t) % 128 == 0 the row GEMM is fused with its reduction and keeps the
+ *     partials on chip. Requests needing more than the array return TP_ENOSPACE before any launch
+ *     (sizes are bounded before they are multiplied, so huge N, h or F cannot wrap the check).
  *   - In TP_OUT_PARTIALS mode the partials are written to out[] (t fp32 [N, h] buffers).
  *   - All calls share the array and it keeps the last call's contents; every call overwrites all
  *     the scratch it reads, so nothing needs clearing. Calls that overlap on the GPU race on it.

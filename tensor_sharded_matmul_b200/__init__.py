@@ -22,7 +22,7 @@ _lib = C.CDLL(LIB_PATH)
 
 # ---- enums (values of include/tp.h) ----------------------------------------------------------
 TP_OK, TP_EINVAL, TP_ESHAPE, TP_EDIVIS, TP_EALIGN, TP_ECUDA, TP_ETIMEOUT, TP_EUNSUPPORTED, TP_ENOSPACE = range(9)
-TP_F32, TP_BF16 = 0, 1
+TP_F32, TP_BF16, TP_BF16_RING = 0, 1, 2
 TP_ACT_NONE, TP_ACT_GELU, TP_ACT_GELU_TANH, TP_ACT_SWIGLU = 0, 1, 2, 3
 TP_OUT_PARTIALS, TP_OUT_RS, TP_OUT_AR, TP_OUT_RS_AG = 0, 1, 2, 3
 TP_CASE1_LOCAL = 0

@@ -37,6 +37,17 @@ RingArgs ring_args(RingOp op, int t, int64_t rows, int64_t cols, int axis, tp_dt
 
 size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
 
+// When the GEMM can read an AllGather's pieces where they lie instead of a gathered copy:
+//   case 2 AllGather (X gathered along D, the contraction): every piece a whole number of 64-wide k-blocks;
+//   case 4 gather X (X gathered along B, rows):             every piece a whole number of 128-row tiles;
+//   case 4 gather W (W gathered along F, columns):          every piece a whole number of 64-wide column boxes.
+bool gather_in_place(int case_id, int strategy, int64_t B, int64_t D, int64_t F, int t) {
+  if (case_id == 2 && strategy == TP_CASE2_ALLGATHER) return D % t == 0 && (D / t) % 64 == 0;
+  if (case_id == 4 && strategy == TP_CASE4_GATHER_X) return B % t == 0 && (B / t) % 128 == 0;
+  if (case_id == 4 && strategy == TP_CASE4_GATHER_W) return F % t == 0 && (F / t) % 64 == 0;
+  return false;
+}
+
 tp_status column_gemm(const uint16_t* x, int64_t N, int64_t k, int64_t n_shard, int t, tp_act act, const uint16_t* w,
                       uint16_t* y, cudaStream_t s) {
   const int64_t wn = act == TP_ACT_SWIGLU ? 2 * n_shard : n_shard;
@@ -243,14 +254,17 @@ size_t tp_sharded_matmul_ws_bytes(int case_id, int strategy, int64_t B, int64_t 
   const size_t T = static_cast<size_t>(t);
   switch (case_id) {
     case 2:   // AllReduce: no workspace when the fused row GEMM + ring reduction applies
-      if (strategy == TP_CASE2_ALLGATHER) return T * align256(size_t(B) * D * 2);
+      if (strategy == TP_CASE2_ALLGATHER)
+        return gather_in_place(case_id, strategy, B, D, F, t) ? 0 : T * align256(size_t(B) * D * 2);
       return (B % t == 0 && ring_gemm_fits(B, F, t, 0)) ? 0 : T * align256(size_t(B) * F * 4);
     case 3: {  // likewise for every case-3 strategy
       const int axis = strategy == TP_CASE3_RS_F ? 1 : 0;
       const bool divides = axis == 1 ? F % t == 0 : B % t == 0;
       return (divides && ring_gemm_fits(B, F, t, axis)) ? 0 : T * align256(size_t(B) * F * 4);
     }
-    case 4: return strategy == TP_CASE4_GATHER_X ? T * align256(size_t(B) * D * 2) : T * align256(size_t(D) * F * 2);
+    case 4:   // no workspace when the GEMM reads the gathered operand's pieces in place
+      if (gather_in_place(case_id, strategy, B, D, F, t)) return 0;
+      return strategy == TP_CASE4_GATHER_X ? T * align256(size_t(B) * D * 2) : T * align256(size_t(D) * F * 2);
     default: return 0;
   }
 }
@@ -282,6 +296,15 @@ tp_status tp_sharded_matmul(int case_id, int strategy, const uint16_t* const* x,
   if (case_id == 2) {                                   // X[B, D_X] . W[D, F]
     if (D % t) return fail(TP_EDIVIS, "t=%d does not divide D", t);
     if (strategy == TP_CASE2_ALLGATHER) {
+      if (gather_in_place(case_id, strategy, B, D, F, t)) {
+        // every shard computes the full C from X's t column pieces, each k-block read from the shard
+        // that holds it: the AllGather is the GEMM's operand addressing
+        GemmArgs g = gemm_args(t, B, F, D, D / t, F, epi);
+        g.a_kslices = t;
+        g.kslice_cols = D / t;
+        for (int i = 0; i < t; ++i) { g.a_kslice[i] = x[i]; g.b[i] = w[i]; g.c[i] = c[i]; }
+        return grouped_gemm(g, s);
+      }
       const size_t slot = align256(size_t(B) * D * 2);
       RingArgs ag = ring_args(RING_AG, t, B, D, 1, TP_BF16, TP_BF16);
       for (int i = 0; i < t; ++i) { ag.in[i] = x[i]; ag.out[i] = wsb + i * slot; }
@@ -336,6 +359,15 @@ tp_status tp_sharded_matmul(int case_id, int strategy, const uint16_t* const* x,
   if (case_id == 4) {                                   // X[B_X, D] . W[D, F_X]: gather one operand
     if (B % t || F % t) return fail(TP_EDIVIS, "t=%d does not divide B and F", t);
     if (strategy == TP_CASE4_GATHER_X) {
+      if (gather_in_place(case_id, strategy, B, D, F, t)) {
+        // shard i multiplies the gathered X by its own columns of W; each 128-row tile of X is read
+        // from the shard that holds it
+        GemmArgs g = gemm_args(t, B, F / t, D, D, F / t, epi);
+        g.a_slices = t;
+        g.slice_rows = B / t;
+        for (int i = 0; i < t; ++i) { g.a_slice[i] = x[i]; g.b[i] = w[i]; g.c[i] = c[i]; }
+        return grouped_gemm(g, s);
+      }
       const size_t slot = align256(size_t(B) * D * 2);
       RingArgs ag = ring_args(RING_AG, t, B, D, 0, TP_BF16, TP_BF16);
       for (int i = 0; i < t; ++i) { ag.in[i] = x[i]; ag.out[i] = wsb + i * slot; }
@@ -345,6 +377,15 @@ tp_status tp_sharded_matmul(int case_id, int strategy, const uint16_t* const* x,
       return grouped_gemm(g, s);
     }
     if (strategy == TP_CASE4_GATHER_W) {
+      if (gather_in_place(case_id, strategy, B, D, F, t)) {
+        // shard i multiplies its rows of X by the gathered W; each 64-column box of W is read from the
+        // shard that holds it
+        GemmArgs g = gemm_args(t, B / t, F, D, D, F / t, epi);
+        g.b_slices = t;
+        g.bslice_cols = F / t;
+        for (int i = 0; i < t; ++i) { g.a[i] = x[i]; g.b_slice[i] = w[i]; g.c[i] = c[i]; }
+        return grouped_gemm(g, s);
+      }
       const size_t slot = align256(size_t(D) * F * 2);
       RingArgs ag = ring_args(RING_AG, t, D, F, 1, TP_BF16, TP_BF16);
       for (int i = 0; i < t; ++i) { ag.in[i] = w[i]; ag.out[i] = wsb + i * slot; }

@@ -14,7 +14,8 @@
 // No atomics, no reassociation, and the result does not depend on grid size.
 // Memory traffic is coalesced 16-byte vectors; grids are a multiple of the SM count with
 // grid-stride loops. bf16 inputs are widened (exact), summed in binary32 and rounded once to bf16
-// (nearest-even) at the end.
+// (nearest-even) at the end; the optional per-hop mode (TP_BF16_RING) instead rounds the running
+// partial to bf16 after every add, as a ring whose links carry bf16 does.
 #include <cuda_bf16.h>
 
 #include <cstring>
@@ -82,6 +83,30 @@ struct IO<uint16_t, 8> {
 };
 
 template <>
+struct IO<float, 4> {
+  static __device__ __forceinline__ void load(const void* base, int64_t i, float (&f)[4]) {
+    const uint4 a = ld_nc_v4(static_cast<const float*>(base) + i);
+    f[0] = __uint_as_float(a.x); f[1] = __uint_as_float(a.y); f[2] = __uint_as_float(a.z); f[3] = __uint_as_float(a.w);
+  }
+  static __device__ __forceinline__ void store(void* base, int64_t i, const float (&f)[4]) {
+    st_v4(static_cast<float*>(base) + i, make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
+                                                    __float_as_uint(f[3])));
+  }
+};
+
+template <>
+struct IO<uint16_t, 4> {
+  static __device__ __forceinline__ void load(const void* base, int64_t i, float (&f)[4]) {
+    const uint2 a = *reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(base) + i);
+    f[0] = __uint_as_float(a.x << 16); f[1] = __uint_as_float(a.x & 0xFFFF0000u);
+    f[2] = __uint_as_float(a.y << 16); f[3] = __uint_as_float(a.y & 0xFFFF0000u);
+  }
+  static __device__ __forceinline__ void store(void* base, int64_t i, const float (&f)[4]) {
+    st_v2(static_cast<uint16_t*>(base) + i, make_uint2(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3])));
+  }
+};
+
+template <>
 struct IO<float, 1> {
   static __device__ __forceinline__ void load(const void* base, int64_t i, float (&f)[1]) {
     f[0] = __ldg(static_cast<const float*>(base) + i);
@@ -114,83 +139,153 @@ __device__ __forceinline__ void locate(const RingParams& p, int64_t e, int& c, i
   }
 }
 
+// The ring sum of the unit starting at full-tensor element e (chunk c) goes out: AllReduce adds the
+// residual (if any) and writes every replica (and the bf16 copy); ReduceScatter writes shard c's
+// piece.
+template <typename Tout, int VEC, bool AR>
+__device__ __forceinline__ void finish_unit(const RingParams& p, int64_t e, int c, float (&acc)[VEC], int t) {
+  if constexpr (AR) {
+    if (p.resid != nullptr) {
+      float r[VEC];
+      if (p.resid_bf16)
+        IO<uint16_t, VEC>::load(p.resid, e, r);
+      else
+        IO<float, VEC>::load(p.resid, e, r);
+#pragma unroll
+      for (int i = 0; i < VEC; ++i) acc[i] = __fadd_rn(acc[i], r[i]);
+    }
+    for (int s = 0; s < t; ++s) IO<Tout, VEC>::store(p.out[s], e, acc);
+    if (p.copy_bf16 != nullptr) IO<uint16_t, VEC>::store(p.copy_bf16, e, acc);
+  } else {
+    int cc;
+    int64_t local;
+    locate(p, e, cc, local);
+    IO<Tout, VEC>::store(p.out[c], local, acc);
+  }
+}
+
+// Round a binary32 value to bfloat16 (nearest-even) and widen it back: one hop of a bf16 ring.
+__device__ __forceinline__ float hop_round(float x) {
+  return __uint_as_float(static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(x))) << 16);
+}
+
 // ReduceScatter (AR == false) or AllReduce (AR == true). TT = compile-time t (0: runtime t).
-template <typename Tin, typename Tout, int VEC, int TT, bool AR>
+// HOP: round the running partial to bf16 after every add (bf16 in and out only).
+// A unit is VEC consecutive elements: one 16-byte vector of the input type (VEC = 1 on the unaligned
+// path), so every warp-wide load is 32 consecutive vectors. A thread takes UNR units per step, a
+// grid stride apart, and issues all their loads before the adds (UNR * t vectors in flight).
+template <typename Tin, typename Tout, int VEC, int TT, bool AR, int UNR, bool HOP>
 __global__ void __launch_bounds__(256) ring_reduce_kernel(const __grid_constant__ RingParams p) {
   const int t = TT > 0 ? TT : p.t;
   const int64_t units = p.rows * p.cols / VEC;
-  for (int64_t u = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; u < units;
-       u += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t e = u * VEC;
-    int c;
-    int64_t local;
-    locate(p, e, c, local);
-    float acc[VEC];
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t u0 = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; u0 < units; u0 += UNR * stride) {
     if constexpr (TT > 0) {
-      float v[TT][VEC];
+      float v[UNR][TT][VEC];
+      int cs[UNR];
 #pragma unroll
-      for (int j = 0; j < TT; ++j) IO<Tin, VEC>::load(p.in[(c + 1 + j) % TT], e, v[j]);   // issue all loads first
+      for (int k = 0; k < UNR; ++k) {
+        const int64_t u = u0 + k * stride;
+        if (u < units) {
+          int64_t local;
+          locate(p, u * VEC, cs[k], local);
 #pragma unroll
-      for (int i = 0; i < VEC; ++i) acc[i] = v[0][i];
+          for (int j = 0; j < TT; ++j) IO<Tin, VEC>::load(p.in[(cs[k] + 1 + j) % TT], u * VEC, v[k][j]);
+        }
+      }
 #pragma unroll
-      for (int j = 1; j < TT; ++j) {
+      for (int k = 0; k < UNR; ++k) {
+        const int64_t u = u0 + k * stride;
+        if (u >= units) break;
+        float acc[VEC];
 #pragma unroll
-        for (int i = 0; i < VEC; ++i) acc[i] = __fadd_rn(acc[i], v[j][i]);
+        for (int i = 0; i < VEC; ++i) acc[i] = v[k][0][i];
+#pragma unroll
+        for (int j = 1; j < TT; ++j) {
+#pragma unroll
+          for (int i = 0; i < VEC; ++i) {
+            acc[i] = __fadd_rn(acc[i], v[k][j][i]);
+            if constexpr (HOP) acc[i] = hop_round(acc[i]);
+          }
+        }
+        finish_unit<Tout, VEC, AR>(p, u * VEC, cs[k], acc, t);
       }
     } else {
-      IO<Tin, VEC>::load(p.in[(c + 1) % t], e, acc);
-      for (int j = 2; j <= t; ++j) {
-        float v[VEC];
-        IO<Tin, VEC>::load(p.in[(c + j) % t], e, v);
+#pragma unroll 1
+      for (int k = 0; k < UNR; ++k) {
+        const int64_t u = u0 + k * stride;
+        if (u >= units) break;
+        const int64_t e = u * VEC;
+        int c;
+        int64_t local;
+        locate(p, e, c, local);
+        float acc[VEC];
+        IO<Tin, VEC>::load(p.in[(c + 1) % t], e, acc);
+        for (int j = 2; j <= t; ++j) {
+          float v[VEC];
+          IO<Tin, VEC>::load(p.in[(c + j) % t], e, v);
 #pragma unroll
-        for (int i = 0; i < VEC; ++i) acc[i] = __fadd_rn(acc[i], v[i]);
+          for (int i = 0; i < VEC; ++i) {
+            acc[i] = __fadd_rn(acc[i], v[i]);
+            if constexpr (HOP) acc[i] = hop_round(acc[i]);
+          }
+        }
+        finish_unit<Tout, VEC, AR>(p, e, c, acc, t);
       }
-    }
-    if constexpr (AR) {
-      if (p.resid != nullptr) {
-        float r[VEC];
-        if (p.resid_bf16)
-          IO<uint16_t, VEC>::load(p.resid, e, r);
-        else
-          IO<float, VEC>::load(p.resid, e, r);
-#pragma unroll
-        for (int i = 0; i < VEC; ++i) acc[i] = __fadd_rn(acc[i], r[i]);
-      }
-      for (int s = 0; s < t; ++s) IO<Tout, VEC>::store(p.out[s], e, acc);
-      if (p.copy_bf16 != nullptr) IO<uint16_t, VEC>::store(p.copy_bf16, e, acc);
-    } else {
-      IO<Tout, VEC>::store(p.out[c], local, acc);
     }
   }
 }
 
 // AllGather as a bit copy: every shard receives every piece. UNIT = bytes moved per step
-// (16 = one vector, or the element size for the unaligned path); ES = element size.
-template <int ES, int UNIT>
+// (16 = one vector, or the element size for the unaligned path); ES = element size. A thread takes
+// UNR units a grid stride apart and loads them all before its stores.
+template <int ES, int UNIT, int UNR>
 __global__ void __launch_bounds__(256) ring_gather_kernel(const __grid_constant__ RingParams p) {
   constexpr int EPU = UNIT / ES;   // elements per unit
   const int64_t units = p.rows * p.cols / EPU;
-  for (int64_t u = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; u < units;
-       u += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t e = u * EPU;
-    int c;
-    int64_t local;
-    locate(p, e, c, local);
-    const char* src = static_cast<const char*>(p.in[c]) + local * ES;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t u0 = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; u0 < units; u0 += UNR * stride) {
     if constexpr (UNIT == 16) {
-      const uint4 v = ld_nc_v4(src);
-      for (int s = 0; s < p.t; ++s) {
-        if (p.skip_self && s == c) continue;
-        st_v4(static_cast<char*>(p.out[s]) + e * ES, v);
+      uint4 v[UNR];
+      int cs[UNR];
+#pragma unroll
+      for (int k = 0; k < UNR; ++k) {
+        const int64_t u = u0 + k * stride;
+        if (u < units) {
+          int64_t local;
+          locate(p, u * EPU, cs[k], local);
+          v[k] = ld_nc_v4(static_cast<const char*>(p.in[cs[k]]) + local * ES);
+        }
       }
-    } else if constexpr (ES == 4) {
-      const uint32_t v = *reinterpret_cast<const uint32_t*>(src);
-      for (int s = 0; s < p.t; ++s)
-        if (!(p.skip_self && s == c)) reinterpret_cast<uint32_t*>(p.out[s])[e] = v;
+#pragma unroll
+      for (int k = 0; k < UNR; ++k) {
+        const int64_t u = u0 + k * stride;
+        if (u >= units) break;
+        for (int s = 0; s < p.t; ++s) {
+          if (p.skip_self && s == cs[k]) continue;
+          st_v4(static_cast<char*>(p.out[s]) + u * EPU * ES, v[k]);
+        }
+      }
     } else {
-      const uint16_t v = *reinterpret_cast<const uint16_t*>(src);
-      for (int s = 0; s < p.t; ++s)
-        if (!(p.skip_self && s == c)) reinterpret_cast<uint16_t*>(p.out[s])[e] = v;
+#pragma unroll 1
+      for (int k = 0; k < UNR; ++k) {
+        const int64_t u = u0 + k * stride;
+        if (u >= units) break;
+        const int64_t e = u * EPU;
+        int c;
+        int64_t local;
+        locate(p, e, c, local);
+        const char* src = static_cast<const char*>(p.in[c]) + local * ES;
+        if constexpr (ES == 4) {
+          const uint32_t v = *reinterpret_cast<const uint32_t*>(src);
+          for (int s = 0; s < p.t; ++s)
+            if (!(p.skip_self && s == c)) reinterpret_cast<uint32_t*>(p.out[s])[e] = v;
+        } else {
+          const uint16_t v = *reinterpret_cast<const uint16_t*>(src);
+          for (int s = 0; s < p.t; ++s)
+            if (!(p.skip_self && s == c)) reinterpret_cast<uint16_t*>(p.out[s])[e] = v;
+        }
+      }
     }
   }
 }
@@ -248,30 +343,54 @@ __global__ void __launch_bounds__(256, 4) all_to_all_kernel(const __grid_constan
   }
 }
 
-int grid_for(int64_t units) {
+// Grid for `units` of work at `unr` units per thread step: at most 8 blocks of 256 threads per SM
+// (a full SM), and no more threads than needed to give every thread the same number of steps, so
+// the last step is not a partial wave.
+int grid_for(int64_t units, int unr) {
   const int sms = sm_count();
-  const int64_t cap = static_cast<int64_t>(sms) * 8;   // 8 x 256 threads: a full SM
-  const int64_t want = (units + 255) / 256;
-  return static_cast<int>(want < cap ? want : cap);
+  const int64_t cap_threads = static_cast<int64_t>(sms) * 8 * 256;
+  const int64_t steps = (units + unr * cap_threads - 1) / (unr * cap_threads);        // per thread
+  const int64_t threads = (units + unr * steps - 1) / (unr * steps);
+  return static_cast<int>((threads + 255) / 256);
 }
 
-template <typename Tin, typename Tout, int VEC, bool AR>
-void launch_reduce(const RingParams& p, int blocks, cudaStream_t s) {
+// Units per thread step: about 8 input vectors in flight per thread.
+template <int TT>
+constexpr int unroll_for() {
+  return TT == 2 ? 4 : TT == 4 ? 2 : 1;
+}
+
+template <typename Tin, typename Tout, int VEC, bool AR, bool HOP = false>
+tp_status launch_reduce(const RingParams& p, int64_t units, cudaStream_t s) {
   switch (p.t) {
-    case 2: ring_reduce_kernel<Tin, Tout, VEC, 2, AR><<<blocks, 256, 0, s>>>(p); break;
-    case 4: ring_reduce_kernel<Tin, Tout, VEC, 4, AR><<<blocks, 256, 0, s>>>(p); break;
-    case 8: ring_reduce_kernel<Tin, Tout, VEC, 8, AR><<<blocks, 256, 0, s>>>(p); break;
-    default: ring_reduce_kernel<Tin, Tout, VEC, 0, AR><<<blocks, 256, 0, s>>>(p); break;
+    case 2: ring_reduce_kernel<Tin, Tout, VEC, 2, AR, unroll_for<2>(), HOP><<<grid_for(units, unroll_for<2>()), 256, 0, s>>>(p); break;
+    case 4: ring_reduce_kernel<Tin, Tout, VEC, 4, AR, unroll_for<4>(), HOP><<<grid_for(units, unroll_for<4>()), 256, 0, s>>>(p); break;
+    case 8: ring_reduce_kernel<Tin, Tout, VEC, 8, AR, 1, HOP><<<grid_for(units, 1), 256, 0, s>>>(p); break;
+    default: ring_reduce_kernel<Tin, Tout, VEC, 0, AR, 1, HOP><<<grid_for(units, 1), 256, 0, s>>>(p); break;
   }
+  return TP_OK;
 }
 
-template <int VEC, bool AR>
-void dispatch_reduce(const RingParams& p, tp_dtype din, tp_dtype dout, int blocks, cudaStream_t s) {
-  if (din == TP_F32 && dout == TP_F32) launch_reduce<float, float, VEC, AR>(p, blocks, s);
-  else if (din == TP_BF16 && dout == TP_BF16) launch_reduce<uint16_t, uint16_t, VEC, AR>(p, blocks, s);
-  else if (din == TP_F32 && dout == TP_BF16) launch_reduce<float, uint16_t, VEC, AR>(p, blocks, s);
-  else launch_reduce<uint16_t, float, VEC, AR>(p, blocks, s);
+// Vector width: one 16-byte vector of the input type (fp32: 4, bf16: 8), or 1 on the unaligned path.
+template <bool AR>
+tp_status dispatch_reduce(const RingParams& p, tp_dtype din, tp_dtype dout, bool vec, cudaStream_t s) {
+  const int64_t n = p.rows * p.cols;
+  if (din == TP_BF16_RING)   // bf16 in and out, the partial rounded after every hop
+    return vec ? launch_reduce<uint16_t, uint16_t, 8, AR, true>(p, n / 8, s)
+               : launch_reduce<uint16_t, uint16_t, 1, AR, true>(p, n, s);
+  if (!vec) {
+    if (din == TP_F32 && dout == TP_F32) return launch_reduce<float, float, 1, AR>(p, n, s);
+    if (din == TP_BF16 && dout == TP_BF16) return launch_reduce<uint16_t, uint16_t, 1, AR>(p, n, s);
+    if (din == TP_F32 && dout == TP_BF16) return launch_reduce<float, uint16_t, 1, AR>(p, n, s);
+    return launch_reduce<uint16_t, float, 1, AR>(p, n, s);
+  }
+  if (din == TP_F32 && dout == TP_F32) return launch_reduce<float, float, 4, AR>(p, n / 4, s);
+  if (din == TP_BF16 && dout == TP_BF16) return launch_reduce<uint16_t, uint16_t, 8, AR>(p, n / 8, s);
+  if (din == TP_F32 && dout == TP_BF16) return launch_reduce<float, uint16_t, 4, AR>(p, n / 4, s);
+  return launch_reduce<uint16_t, float, 8, AR>(p, n / 8, s);
 }
+
+bool ring_dtype_ok(tp_dtype d) { return d == TP_F32 || d == TP_BF16 || d == TP_BF16_RING; }
 
 }  // namespace
 
@@ -280,8 +399,9 @@ tp_status ring_collective(const RingArgs& a, cudaStream_t stream) {
   if (a.rows < 0 || a.cols < 0) return fail(TP_EINVAL, "negative size");
   if (a.rows == 0 || a.cols == 0) return TP_OK;         // empty buffers: nothing to move
   if (a.axis != 0 && a.axis != 1) return fail(TP_EINVAL, "axis must be 0 or 1");
-  if ((a.in_dtype != TP_F32 && a.in_dtype != TP_BF16) || (a.out_dtype != TP_F32 && a.out_dtype != TP_BF16))
-    return fail(TP_EINVAL, "bad dtype");
+  const bool hop = a.in_dtype == TP_BF16_RING || a.out_dtype == TP_BF16_RING;
+  if (hop && a.in_dtype != a.out_dtype) return fail(TP_EINVAL, "per-hop bf16 rounding needs bf16 in and out");
+  if (!ring_dtype_ok(a.in_dtype) || !ring_dtype_ok(a.out_dtype)) return fail(TP_EINVAL, "bad dtype");
   if (a.op == RING_AG && a.in_dtype != a.out_dtype) return fail(TP_EINVAL, "AllGather copies bits: dtypes must match");
   const int axis = a.op == RING_AR ? 0 : a.axis;
   if (axis == 0 && a.rows % a.t) return fail(TP_EDIVIS, "t=%d does not divide rows=%lld", a.t, (long long)a.rows);
@@ -308,7 +428,7 @@ tp_status ring_collective(const RingArgs& a, cudaStream_t stream) {
   const int sms = sm_count();
   if (sms <= 0) return fail(TP_ECUDA, "cannot query the SM count");
 
-  if (a.op == RING_AG) {
+  if (a.op == RING_AG) {   // a bit copy: TP_BF16_RING moves bf16 like TP_BF16
     const int es = a.in_dtype == TP_F32 ? 4 : 2;
     const int epu = 16 / es;
     bool vec = all16 && (axis == 0 ? p.chunk_elems % epu == 0 : (p.chunk_cols % epu == 0 && a.cols % epu == 0));
@@ -318,28 +438,23 @@ tp_status ring_collective(const RingArgs& a, cudaStream_t stream) {
       in_place = static_cast<const char*>(a.in[i]) == static_cast<const char*>(a.out[i]) + i * p.chunk_elems * es;
     p.skip_self = in_place ? 1 : 0;
     const int64_t units = a.rows * a.cols / (vec ? epu : 1);
-    const int blocks = grid_for(units);
+    constexpr int G_UNR = 2;
+    const int blocks = grid_for(units, G_UNR);
     if (es == 4) {
-      if (vec) ring_gather_kernel<4, 16><<<blocks, 256, 0, stream>>>(p);
-      else ring_gather_kernel<4, 4><<<blocks, 256, 0, stream>>>(p);
+      if (vec) ring_gather_kernel<4, 16, G_UNR><<<blocks, 256, 0, stream>>>(p);
+      else ring_gather_kernel<4, 4, G_UNR><<<blocks, 256, 0, stream>>>(p);
     } else {
-      if (vec) ring_gather_kernel<2, 16><<<blocks, 256, 0, stream>>>(p);
-      else ring_gather_kernel<2, 2><<<blocks, 256, 0, stream>>>(p);
+      if (vec) ring_gather_kernel<2, 16, G_UNR><<<blocks, 256, 0, stream>>>(p);
+      else ring_gather_kernel<2, 2, G_UNR><<<blocks, 256, 0, stream>>>(p);
     }
     return check_launch("ring_gather_kernel");
   }
 
-  // Vectors of 8 elements must not straddle a chunk (or, for axis 1, a row).
+  // A unit (one 16-byte vector of the input type) must not straddle a chunk (or, for axis 1, a row).
+  // Checking multiples of 8 elements covers both vector widths (4 fp32, 8 bf16).
   const bool vec = all16 && (axis == 0 ? p.chunk_elems % 8 == 0 : (p.chunk_cols % 8 == 0 && a.cols % 8 == 0));
-  const int64_t units = a.rows * a.cols / (vec ? 8 : 1);
-  const int blocks = grid_for(units);
-  if (a.op == RING_RS) {
-    if (vec) dispatch_reduce<8, false>(p, a.in_dtype, a.out_dtype, blocks, stream);
-    else dispatch_reduce<1, false>(p, a.in_dtype, a.out_dtype, blocks, stream);
-  } else {
-    if (vec) dispatch_reduce<8, true>(p, a.in_dtype, a.out_dtype, blocks, stream);
-    else dispatch_reduce<1, true>(p, a.in_dtype, a.out_dtype, blocks, stream);
-  }
+  if (a.op == RING_RS) dispatch_reduce<false>(p, a.in_dtype, a.out_dtype, vec, stream);
+  else dispatch_reduce<true>(p, a.in_dtype, a.out_dtype, vec, stream);
   return check_launch("ring_reduce_kernel");
 }
 

@@ -65,6 +65,17 @@ struct GemmArgs {
   int a_slices;
   int64_t slice_rows;
   const uint16_t* a_slice[TP_MAX_SHARDS];
+  // Optional: A given as a_kslices column slices [M, kslice_cols] (row stride lda) shared by every
+  // group (a[] is then ignored); column k of A is column k % kslice_cols of a_kslice[k / kslice_cols]
+  // (an AllGather along the contraction, read where each piece lies).
+  int a_kslices;
+  int64_t kslice_cols;
+  const uint16_t* a_kslice[TP_MAX_SHARDS];
+  // Optional: B given as b_slices column slices [K, bslice_cols] (row stride ldb) shared by every
+  // group (b[] is then ignored); column n of B is column n % bslice_cols of b_slice[n / bslice_cols].
+  int b_slices;
+  int64_t bslice_cols;
+  const uint16_t* b_slice[TP_MAX_SHARDS];
   // Transposed storage: a_mn = A given as A^T [K][M] (row stride lda >= M); b_km = B given as
   // B^T [N][K] (row stride ldb >= K).
   bool a_mn, b_km;

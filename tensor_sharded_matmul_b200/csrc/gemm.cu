@@ -143,11 +143,28 @@ __device__ __forceinline__ void init_barriers(const Ctl& c, uint32_t epilogue_wa
   fence_mbar_init();
 }
 
+// Operand pieces of a sliced operand: the view that holds element `x` of the sliced dimension, and
+// x's place inside it. Past the last piece the last view is used with an out-of-range coordinate,
+// which TMA fills with zeros (the padding k-block of an odd k-block count, a partial last tile).
+__device__ __forceinline__ const CUtensorMap* slice_view(const CUtensorMap* base, int width, int count, int x, int& lx) {
+  if (width == 0) {
+    lx = x;
+    return base;
+  }
+  int sl = x / width;
+  if (sl > count - 1) sl = count - 1;
+  lx = x - sl * width;
+  return base + sl;
+}
+
 // Producer: the num_kb k-blocks of one unit. B is four 64-wide boxes of `b` at n0 (b2 == nullptr),
-// or two boxes of `b` and two of `b2`, both at n0 (SwiGLU: gate and up halves).
+// or two boxes of `b` and two of `b2`, both at n0 (SwiGLU: gate and up halves). a_kslice != 0: A is
+// a_kslices views of a_kslice columns each, starting at `a` (A split along K). b_nslice != 0: B is
+// b_nslices views of b_nslice columns each, starting at `b` (B split along N).
 __device__ __forceinline__ bool produce_unit(const Ctl& c, Ring& r, const CUtensorMap* a, const CUtensorMap* b,
                                              const CUtensorMap* b2, int m0, int n0, int num_kb, int* last_phase,
-                                             bool* issued) {
+                                             bool* issued, int a_kslice = 0, int a_kslices = 1, int b_nslice = 0,
+                                             int b_nslices = 1) {
   for (int kb = 0; kb < num_kb; ++kb) {
     if (!wait_or_abort(c, c.empty0 + 8 * r.stage, r.phase ^ 1u, WAIT_PRODUCER_EMPTY)) return false;
     const uint32_t fb = c.full0 + 8 * r.stage;
@@ -159,7 +176,9 @@ __device__ __forceinline__ bool produce_unit(const Ctl& c, Ring& r, const CUtens
       tma_load_2d(a_dst, a, m0, k0, fb);
       tma_load_2d(a_dst + B_BOX, a, m0 + 64, k0, fb);
     } else {                            // A [M][K]: one 64(K) x 128(M) box
-      tma_load_2d(a_dst, a, k0, m0, fb);
+      int ak0;
+      const CUtensorMap* av = slice_view(a, a_kslice, a_kslices, k0, ak0);
+      tma_load_2d(a_dst, av, ak0, m0, fb);
     }
     // B (the weights) is re-read by every row-tile: the fused kernel keeps its lines in L2 longest
     if (c.b_km) {                       // B^T [N][K]: one 64(K) x 256(N) box
@@ -171,7 +190,11 @@ __device__ __forceinline__ bool produce_unit(const Ctl& c, Ring& r, const CUtens
       tma_load_2d_hint(b_dst + 3 * B_BOX, b2, n0 + 64, k0, fb, c.b_policy);
     } else {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) tma_load_2d_hint(b_dst + j * B_BOX, b, n0 + 64 * j, k0, fb, c.b_policy);
+      for (int j = 0; j < 4; ++j) {
+        int bn;
+        const CUtensorMap* bv = slice_view(b, b_nslice, b_nslices, n0 + 64 * j, bn);
+        tma_load_2d_hint(b_dst + j * B_BOX, bv, bn, k0, fb, c.b_policy);
+      }
     }
     issued[r.stage] = true;
     last_phase[r.stage] = static_cast<int>(r.phase);
@@ -282,6 +305,13 @@ struct GemmParams {
   // A given as row slices shared by all groups (the sequence-parallel entry: A = AllGather of t
   // row shards): row m of A is row m % slice_rows of ta[m / slice_rows]. 0 = one A per group.
   int a_slices, slice_rows;
+  // A given as a_kslices column slices of a_kslice columns shared by all groups (the AllGather along
+  // the contraction): column k of A is column k % a_kslice of ta[k / a_kslice]. 0 = not sliced.
+  int a_kslice, a_kslices;
+  // B given as b_nslices column slices of b_nslice columns shared by all groups (the AllGather of a
+  // column-split weight): column n of B is column n % b_nslice of tb[n / b_nslice]. 0 = not sliced.
+  int b_nslice, b_nslices;
+  int n_amaps, n_bmaps;             // tensor maps in ta[] / tb[] (prefetched at start)
   bool a_mn, b_km;                  // A stored [K][M] / B stored [N][K] (transposed operands)
   uint32_t* status;
   unsigned long long budget;
@@ -289,6 +319,10 @@ struct GemmParams {
 
 // Tensor map and local row of A for a tile starting at row m0 of group g.
 __device__ __forceinline__ const CUtensorMap* a_view(const GemmParams& p, int g, int m0, int& am0) {
+  if (p.a_kslice) {                 // every group reads the same K slices (chosen per k-block)
+    am0 = m0;
+    return &p.ta[0];
+  }
   if (p.a_slices) {
     const int sl = m0 / p.slice_rows;
     am0 = m0 - sl * p.slice_rows;
@@ -340,11 +374,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tcgen05_kernel(const __g
 
   if (threadIdx.x == 0) init_barriers(c, 4);
   if (warp == 0 && lane == 0) {
-    for (int g = 0; g < p.groups; ++g) {
+    for (int g = 0; g < p.n_bmaps; ++g) {
       prefetch_tmap(&p.tb[g]);
       if (SWIGLU) prefetch_tmap(&p.tb2[g]);
     }
-    for (int g = 0; g < (p.a_slices ? p.a_slices : p.groups); ++g) prefetch_tmap(&p.ta[g]);
+    for (int g = 0; g < p.n_amaps; ++g) prefetch_tmap(&p.ta[g]);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
@@ -371,8 +405,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tcgen05_kernel(const __g
         const int m0 = (rt - g * p.tiles_m) * BM;
         int am0;
         const CUtensorMap* ta = a_view(p, g, m0, am0);
-        if (!produce_unit(c, r, ta, &p.tb[g], SWIGLU ? &p.tb2[g] : nullptr, am0, nt * TILE_N, p.num_kb,
-                          last_phase, issued))
+        if (!produce_unit(c, r, ta, p.b_nslice ? &p.tb[0] : &p.tb[g], SWIGLU ? &p.tb2[g] : nullptr, am0,
+                          nt * TILE_N, p.num_kb, last_phase, issued, p.a_kslice, p.a_kslices, p.b_nslice,
+                          p.b_nslices))
           break;
       }
     }
@@ -510,7 +545,9 @@ __device__ __forceinline__ bool pair_fail(const PairCtl& c, uint32_t site) {
 // zeros and is not multiplied). m0 is this CTA's first row, nb its first B column: two 64-wide boxes
 // of `tb` per k-block for a full tile, one for a half-width tile (wide == false, B stored [K][N] only).
 __device__ __forceinline__ bool pair_produce_unit(const PairCtl& c, PairRing& r, const CUtensorMap* ta, int m0,
-                                                  const CUtensorMap* tb, int nb, int num_kb, bool wide = true) {
+                                                  const CUtensorMap* tb, int nb, int num_kb, bool wide = true,
+                                                  int a_kslice = 0, int a_kslices = 1, int b_nslice = 0,
+                                                  int b_nslices = 1) {
   const uint32_t tx = 2 * (PAIR_A_STAGE + (wide ? PAIR_B_STAGE : PAIR_B_STAGE / 2));
   for (int kb = 0; kb < num_kb; kb += PAIR_KB) {
     if (!mbar_wait_bounded(c.empty0 + 8 * r.stage, r.phase ^ 1u, c.budget, c.abort_flag))
@@ -526,13 +563,20 @@ __device__ __forceinline__ bool pair_produce_unit(const PairCtl& c, PairRing& r,
         tma_load_2d_pair(a_dst, ta, m0, k0, fb);
         tma_load_2d_pair(a_dst + B_BOX, ta, m0 + 64, k0, fb);
       } else {
-        tma_load_2d_pair(a_dst, ta, k0, m0, fb);
+        int ak0;
+        const CUtensorMap* av = slice_view(ta, a_kslice, a_kslices, k0, ak0);
+        tma_load_2d_pair(a_dst, av, ak0, m0, fb);
       }
       if (c.b_km) {                     // B^T [N][K]: one 64(K) x 128(N) box of this CTA's columns
         tma_load_2d_pair_hint(b_dst, tb, k0, nb, fb, c.b_policy);
       } else {
-        tma_load_2d_pair_hint(b_dst, tb, nb, k0, fb, c.b_policy);
-        if (wide) tma_load_2d_pair_hint(b_dst + B_BOX, tb, nb + 64, k0, fb, c.b_policy);
+        int bn;
+        const CUtensorMap* bv = slice_view(tb, b_nslice, b_nslices, nb, bn);
+        tma_load_2d_pair_hint(b_dst, bv, bn, k0, fb, c.b_policy);
+        if (wide) {
+          bv = slice_view(tb, b_nslice, b_nslices, nb + 64, bn);
+          tma_load_2d_pair_hint(b_dst + B_BOX, bv, bn, k0, fb, c.b_policy);
+        }
       }
     }
     r.advance();
@@ -629,11 +673,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
   if (warp == 0 && lane == 0) {
-    for (int g = 0; g < p.groups; ++g) {
+    for (int g = 0; g < p.n_bmaps; ++g) {
       prefetch_tmap(&p.tb[g]);
       if (SWIGLU) prefetch_tmap(&p.tb2[g]);
     }
-    for (int g = 0; g < (p.a_slices ? p.a_slices : p.groups); ++g) prefetch_tmap(&p.ta[g]);
+    for (int g = 0; g < p.n_amaps; ++g) prefetch_tmap(&p.ta[g]);
   }
   uint32_t* tmem_slot;
   const PairCtl c = pair_setup(smem, 0, tmem_slot, 4, p.status, p.budget, false, p.a_mn, p.b_km);
@@ -654,11 +698,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
         const int g = rt / tiles_m;
         const int m0 = (rt - g * tiles_m) * TILE_M + static_cast<int>(c.rank) * BM;
         const int n0 = nt * TILE_N;
-        const CUtensorMap* tb = SWIGLU ? (c.rank == 0 ? &p.tb[g] : &p.tb2[g]) : &p.tb[g];
+        const CUtensorMap* tb = SWIGLU ? (c.rank == 0 ? &p.tb[g] : &p.tb2[g]) : p.b_nslice ? &p.tb[0] : &p.tb[g];
         const int nb = SWIGLU ? n0 : n0 + static_cast<int>(c.rank) * 128;
         int am0;
         const CUtensorMap* ta = a_view(p, g, m0, am0);
-        if (!pair_produce_unit(c, r, ta, am0, tb, nb, p.num_kb)) break;
+        if (!pair_produce_unit(c, r, ta, am0, tb, nb, p.num_kb, true, p.a_kslice, p.a_kslices, p.b_nslice,
+                               p.b_nslices))
+          break;
       }
     }
   } else if (warp == 1) {
@@ -1196,13 +1242,16 @@ tp_status grouped_gemm(const GemmArgs& g, cudaStream_t s) {
   if (g.M == 0 || g.N == 0) return TP_OK;               // empty output: nothing to compute
   if (g.M > INT32_MAX / 2 || g.N > INT32_MAX / 2 || g.K > INT32_MAX / 2) return fail(TP_ESHAPE, "GEMM size too large");
   const bool swiglu = g.epi == EPI_SWIGLU;
+  const bool a_sliced = g.a_slices || g.a_kslices;
   if (g.K % 8 || g.N % 8 || g.lda % 8 || g.ldb % 8) return fail(TP_EALIGN, "K, N and row strides must be multiples of 8");
   if (g.M % 8 && g.a_mn) return fail(TP_EALIGN, "M must be a multiple of 8 for a transposed A");
-  if (g.lda < (g.a_mn ? g.M : g.K) || g.ldb < (g.b_km ? g.K : (swiglu ? 2 * g.N : g.N)))
-    return fail(TP_ESHAPE, "row stride shorter than the row");
+  const int64_t a_row = g.a_kslices ? g.kslice_cols : (g.a_mn ? g.M : g.K);
+  const int64_t b_row = g.b_slices ? g.bslice_cols : (g.b_km ? g.K : (swiglu ? 2 * g.N : g.N));
+  if (g.lda < a_row || g.ldb < b_row) return fail(TP_ESHAPE, "row stride shorter than the row");
   for (int i = 0; i < g.groups; ++i) {
-    if ((!g.a_slices && g.a[i] == nullptr) || g.b[i] == nullptr || g.c[i] == nullptr) return fail(TP_EINVAL, "null GEMM operand %d", i);
-    if ((!g.a_slices && !aligned16(g.a[i])) || !aligned16(g.b[i]) || !aligned16(g.c[i]))
+    if ((!a_sliced && g.a[i] == nullptr) || (!g.b_slices && g.b[i] == nullptr) || g.c[i] == nullptr)
+      return fail(TP_EINVAL, "null GEMM operand %d", i);
+    if ((!a_sliced && !aligned16(g.a[i])) || (!g.b_slices && !aligned16(g.b[i])) || !aligned16(g.c[i]))
       return fail(TP_EALIGN, "GEMM operand %d not 16-byte aligned", i);
   }
   GemmParams p;
@@ -1210,6 +1259,8 @@ tp_status grouped_gemm(const GemmArgs& g, cudaStream_t s) {
   const int tile_n = swiglu ? BN / 2 : BN;
   const bool pair = g.M >= 2 * BM && (g.a_slices == 0 || g.slice_rows % (2 * BM) == 0);
   if (g.a_slices && g.a_mn) return fail(TP_EUNSUPPORTED, "row slices of a transposed A are not supported");
+  if (g.a_kslices && (g.a_mn || g.a_slices)) return fail(TP_EUNSUPPORTED, "K slices need A as [M][K] and no row slices");
+  if (g.b_slices && (g.b_km || swiglu)) return fail(TP_EUNSUPPORTED, "column slices need B as [K][N], no SwiGLU");
   if (swiglu && g.b_km) return fail(TP_EUNSUPPORTED, "SwiGLU needs B as [K][2N]");
   if (g.a_slices) {
     if (g.a_slices > TP_MAX_SHARDS || g.slice_rows <= 0 || g.slice_rows % BM != 0 || g.slice_rows * g.a_slices != g.M)
@@ -1223,13 +1274,40 @@ tp_status grouped_gemm(const GemmArgs& g, cudaStream_t s) {
     p.a_slices = g.a_slices;
     p.slice_rows = static_cast<int>(g.slice_rows);
   }
+  if (g.a_kslices) {   // A split along K: each k-block is read from the piece that holds it
+    if (g.a_kslices > TP_MAX_SHARDS || g.kslice_cols <= 0 || g.kslice_cols % BK != 0 || g.kslice_cols * g.a_kslices != g.K)
+      return fail(TP_ESHAPE, "A's K slices must tile K in multiples of %d columns", BK);
+    for (int i = 0; i < g.a_kslices; ++i) {
+      if (g.a_kslice[i] == nullptr) return fail(TP_EINVAL, "null A K slice %d", i);
+      if (!aligned16(g.a_kslice[i])) return fail(TP_EALIGN, "A K slice %d not 16-byte aligned", i);
+      if (!encode_bf16_2d(&p.ta[i], g.a_kslice[i], g.kslice_cols, g.M, g.lda, BK, BM))
+        return fail(TP_ECUDA, "cannot encode the TMA descriptor of A K slice %d", i);
+    }
+    p.a_kslice = static_cast<int>(g.kslice_cols);
+    p.a_kslices = g.a_kslices;
+  }
+  if (g.b_slices) {    // B split along N: each 64-column box is read from the piece that holds it
+    if (g.b_slices > TP_MAX_SHARDS || g.bslice_cols <= 0 || g.bslice_cols % 64 != 0 || g.bslice_cols * g.b_slices != g.N)
+      return fail(TP_ESHAPE, "B's column slices must tile N in multiples of 64 columns");
+    for (int i = 0; i < g.b_slices; ++i) {
+      if (g.b_slice[i] == nullptr) return fail(TP_EINVAL, "null B column slice %d", i);
+      if (!aligned16(g.b_slice[i])) return fail(TP_EALIGN, "B column slice %d not 16-byte aligned", i);
+      if (!encode_bf16_2d(&p.tb[i], g.b_slice[i], g.bslice_cols, g.K, g.ldb, 64, BK))
+        return fail(TP_ECUDA, "cannot encode the TMA descriptor of B column slice %d", i);
+    }
+    p.b_nslice = static_cast<int>(g.bslice_cols);
+    p.b_nslices = g.b_slices;
+  }
+  p.n_amaps = g.a_slices ? g.a_slices : g.a_kslices ? g.a_kslices : g.groups;
+  p.n_bmaps = g.b_slices ? g.b_slices : g.groups;
   for (int i = 0; i < g.groups; ++i) {
-    const bool a_ok = g.a_slices ? true
+    const bool a_ok = a_sliced ? true
                       : g.a_mn ? encode_bf16_2d(&p.ta[i], g.a[i], g.M, g.K, g.lda, 64, BK)
                                : encode_bf16_2d(&p.ta[i], g.a[i], g.K, g.M, g.lda, BK, BM);
     if (!a_ok) return fail(TP_ECUDA, "cannot encode the TMA descriptor of A[%d]", i);
-    const bool b_ok = g.b_km ? encode_bf16_2d(&p.tb[i], g.b[i], g.K, g.N, g.ldb, BK, pair ? 128 : BN)
-                             : encode_bf16_2d(&p.tb[i], g.b[i], g.N, g.K, g.ldb, 64, BK);
+    const bool b_ok = g.b_slices ? true
+                      : g.b_km ? encode_bf16_2d(&p.tb[i], g.b[i], g.K, g.N, g.ldb, BK, pair ? 128 : BN)
+                               : encode_bf16_2d(&p.tb[i], g.b[i], g.N, g.K, g.ldb, 64, BK);
     if (!b_ok) return fail(TP_ECUDA, "cannot encode the TMA descriptor of B[%d]", i);
     if (swiglu && !encode_bf16_2d(&p.tb2[i], g.b[i] + g.N, g.N, g.K, g.ldb, 64, BK))
       return fail(TP_ECUDA, "cannot encode the TMA descriptor of the up half of B[%d]", i);
@@ -1313,7 +1391,8 @@ tp_status ring_gemm(const RingGemmArgs& g, cudaStream_t s) {
   p.chunk = static_cast<int>(axis == 0 ? g.M / g.t : g.N / g.t);
   // CTA pairs when every chunk is a whole number of 256-row (axis 0) or 256-column (axis 1) tiles
   p.chunk_tiles = axis == 0 ? p.chunk / (pair ? 2 * BM : BM) : p.chunk / BN;
-  p.tiles_m = static_cast<int>(g.M / BM);
+  // axis 0 has M a multiple of 128 (whole-tile chunks); axis 1 may end in a partial row-tile
+  p.tiles_m = static_cast<int>((g.M + BM - 1) / BM);
   p.tiles_n = static_cast<int>((g.N + BN - 1) / BN);
   p.num_tiles = p.tiles_m * p.tiles_n;
   p.num_kb = static_cast<int>((g.K + BK - 1) / BK);

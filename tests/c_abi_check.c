@@ -32,6 +32,7 @@ int main(void) {
                                                           c4, TP_F32, NULL, 0, NULL));
   /* workspace sizes (host arithmetic) */
   printf("ws_case4_gather_w %zu\n", tp_sharded_matmul_ws_bytes(4, TP_CASE4_GATHER_W, 8192, 8192, 28672, 4));
+  printf("ws_case4_gather_w_ragged %zu\n", tp_sharded_matmul_ws_bytes(4, TP_CASE4_GATHER_W, 8192, 8192, 384, 4));
   printf("ws_case3_fused %zu\n", tp_sharded_matmul_ws_bytes(3, TP_CASE3_RS_B, 8192, 8192, 28672, 4));
   return 0;
 }

@@ -92,7 +92,15 @@ def test_gemm_and_mlp_validate_before_launch():
 def test_sharded_matmul_workspace_sizes_and_validation():
     B, D, F, t = 8192, 8192, 28672, 4
     assert tp.tp_sharded_matmul_ws_bytes(1, 0, B, D, F, t) == 0
-    assert tp.tp_sharded_matmul_ws_bytes(2, tp.TP_CASE2_ALLGATHER, B, D, F, t) == t * B * D * 2
+    # the gathering strategies read the gathered operand's pieces in place when they are whole
+    # 64-wide k-blocks (case 2), 128-row tiles (case 4, X) or 64-column boxes (case 4, W) ...
+    assert tp.tp_sharded_matmul_ws_bytes(2, tp.TP_CASE2_ALLGATHER, B, D, F, t) == 0
+    assert tp.tp_sharded_matmul_ws_bytes(4, tp.TP_CASE4_GATHER_X, B, D, F, t) == 0
+    assert tp.tp_sharded_matmul_ws_bytes(4, tp.TP_CASE4_GATHER_W, B, D, F, t) == 0
+    # ... and materialise the gather otherwise (one gathered copy per shard)
+    assert tp.tp_sharded_matmul_ws_bytes(2, tp.TP_CASE2_ALLGATHER, B, 96 * 4, F, t) == t * B * 384 * 2
+    assert tp.tp_sharded_matmul_ws_bytes(4, tp.TP_CASE4_GATHER_X, 64 * 4, D, F, t) == t * 256 * D * 2
+    assert tp.tp_sharded_matmul_ws_bytes(4, tp.TP_CASE4_GATHER_W, B, D, 96 * 4, t) == t * D * 384 * 2
     # the fused row GEMM + ring reduction needs no workspace when the chunks are whole tiles ...
     assert tp.tp_sharded_matmul_ws_bytes(2, tp.TP_CASE2_ALLREDUCE, B, D, F, t) == 0
     assert tp.tp_sharded_matmul_ws_bytes(3, tp.TP_CASE3_RS_F, B, D, F, t) == 0
@@ -101,7 +109,6 @@ def test_sharded_matmul_workspace_sizes_and_validation():
     assert tp.tp_sharded_matmul_ws_bytes(2, tp.TP_CASE2_ALLREDUCE, 96, D, F, t) == t * 96 * F * 4
     assert tp.tp_sharded_matmul_ws_bytes(3, tp.TP_CASE3_RS_B, 96, D, F, t) == t * 96 * F * 4
     assert tp.tp_sharded_matmul_ws_bytes(3, tp.TP_CASE3_RS_F, B, D, 1000, t) == t * B * 1000 * 4
-    assert tp.tp_sharded_matmul_ws_bytes(4, tp.TP_CASE4_GATHER_W, B, D, F, t) == t * D * F * 2
     _expect(tp.TP_ENOSPACE, tp.tp_sharded_matmul, 3, 0, [FAKE] * 4, [FAKE] * 4, 64, 64, 64, 4, [FAKE] * 4, tp.TP_F32,
             FAKE, 10, 0)
     _expect(tp.TP_EINVAL, tp.tp_sharded_matmul, 5, 0, [FAKE] * 4, [FAKE] * 4, 64, 64, 64, 4, [FAKE] * 4, tp.TP_F32,
@@ -156,3 +163,29 @@ def test_oversized_problems_are_rejected_before_launch():
     _expect(tp.TP_EDIVIS, tp.tp_reduce_scatter, [FAKE] * 16, [FAKE] * 16, 24, 16, 0, tp.TP_F32, 16, 0)
     _expect(tp.TP_EINVAL, tp.tp_mlp_fwd, FAKE, 64, 256, 1024, 17, tp.TP_ACT_GELU, FAKE, FAKE, FAKE, [FAKE] * 17,
             tp.TP_OUT_PARTIALS, None, 0)
+
+
+def test_noalloc_scratch_bound_cannot_wrap():
+    """tp_mlp_fwd_noalloc bounds every size before multiplying it: sizes whose byte counts would wrap
+    a 64-bit product (and so slip past a check done after the multiplication) give TP_ENOSPACE on
+    the host, before the scratch array is looked up or anything is launched."""
+    huge = 1 << 62
+    A = tp.TP_ACT_GELU
+    # the activations' N*F*2 alone would wrap
+    _expect(tp.TP_ENOSPACE, tp.tp_mlp_fwd_noalloc, FAKE, huge, 256, 8, 4, A, FAKE, FAKE, tp.TP_OUT_PARTIALS, [FAKE] * 4, 0)
+    _expect(tp.TP_ENOSPACE, tp.tp_mlp_fwd_noalloc, FAKE, 8, 256, huge, 4, A, FAKE, FAKE, tp.TP_OUT_AR, [FAKE] * 4, 0)
+    # small Z, but the unfused path's t*N*h*4 partials would wrap (N/t = 1 row: not fusable)
+    _expect(tp.TP_ENOSPACE, tp.tp_mlp_fwd_noalloc, FAKE, 4, huge, 8, 4, A, FAKE, FAKE, tp.TP_OUT_AR, [FAKE] * 4, 0)
+    # in range but larger than the array
+    _expect(tp.TP_ENOSPACE, tp.tp_mlp_fwd_noalloc, FAKE, 4096, 4096, 14336, 8, tp.TP_ACT_SWIGLU, FAKE, FAKE,
+            tp.TP_OUT_PARTIALS, [FAKE] * 8, 0)
+
+
+def test_per_hop_bf16_is_a_ring_collective_mode_only():
+    """TP_BF16_RING is accepted by the ring collectives and refused elsewhere, on the host."""
+    _expect(tp.TP_EINVAL, tp.tp_grouped_gemm, 1, [FAKE], [FAKE], [FAKE], 64, 64, 64, tp.TP_ACT_NONE, tp.TP_BF16_RING, 0)
+    _expect(tp.TP_EINVAL, tp.tp_all_to_all, [FAKE] * 2, [FAKE] * 2, 16, 16, 0, 1, tp.TP_BF16_RING, 2, 0)
+    _expect(tp.TP_EINVAL, tp.tp_reduce_scatter, [FAKE] * 2, [FAKE] * 2, 16, 16, 0, 3, 2, 0)   # unknown dtype
+    # empty inputs pass validation in the per-hop mode like in the others
+    tp.tp_reduce_scatter([0, 0], [0, 0], 0, 16, 0, tp.TP_BF16_RING, 2, 0)
+    tp.tp_all_reduce([0, 0], [0, 0], 0, 16, tp.TP_BF16_RING, 2, 0)

@@ -43,5 +43,6 @@ def test_empty_inputs_and_validation_from_c(c_output):
 
 
 def test_workspace_sizes_from_c(c_output):
-    assert int(c_output["ws_case4_gather_w"]) == 4 * 8192 * 28672 * 2
+    assert int(c_output["ws_case4_gather_w"]) == 0                 # W's pieces read in place
+    assert int(c_output["ws_case4_gather_w_ragged"]) == 4 * 8192 * 384 * 2   # F/t = 96: gathered copy
     assert int(c_output["ws_case3_fused"]) == 0

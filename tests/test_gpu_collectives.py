@@ -27,6 +27,8 @@ CASES = [
     (8, 64, 1024, "f32", 1), (3, 96, 72, "f32", 0), (5, 40, 80, "bf16", 1), (16, 64, 128, "bf16", 0),
     (2, 6, 5, "f32", 0), (3, 9, 7, "bf16", 0), (4, 12, 20, "f32", 1), (2, 10, 3, "bf16", 0),
     (4, 256, 2048, "bf16", 0), (8, 512, 4096, "bf16", 1),
+    # more than one grid-stride step per thread, with the last step of some threads partial
+    (2, 2050, 4104, "f32", 0), (4, 1028, 4104, "bf16", 0), (2, 2050, 4104, "bf16", 1),
 ]
 
 
@@ -210,3 +212,46 @@ def test_all_to_all_moves_the_sharded_dim():
     torch.cuda.synchronize()
     for j in range(t):
         assert torch.equal(outs[j].cpu(), A[:, j * J // t:(j + 1) * J // t])
+
+
+# ---------------------------------------------------------------------------------- per-hop bf16 mode
+@pytest.mark.parametrize("t,rows,cols,axis", [(2, 64, 256, 0), (3, 96, 72, 0), (4, 64, 256, 1), (8, 512, 4096, 0),
+                                              (5, 40, 80, 1), (3, 9, 7, 0), (4, 1028, 4104, 0)])
+def test_per_hop_bf16_reduce_scatter_and_all_reduce_bit_exact(t, rows, cols, axis):
+    ins = _payload(t, rows, cols, "bf16", seed=900 + t * rows + cols)
+    d_in = [cuda(x) for x in ins]
+    oshape = (rows // t, cols) if axis == 0 else (rows, cols // t)
+    rs = [torch.empty(oshape, dtype=torch.bfloat16, device="cuda") for _ in range(t)]
+    tp.tp_reduce_scatter(d_in, rs, rows, cols, axis, tp.TP_BF16_RING, t)
+    ar = [torch.empty((rows, cols), dtype=torch.bfloat16, device="cuda") for _ in range(t)]
+    if axis == 0:
+        tp.tp_all_reduce(d_in, ar, rows, cols, tp.TP_BF16_RING, t)
+    torch.cuda.synchronize()
+    bits = [host_bits(x) for x in ins]
+    ref = OC.reduce_scatter(bits, axis=axis, dtype="bf16", rounding="hop")
+    for r in range(t):
+        assert same_bits(host_bits(rs[r]), ref[r]), f"RS shard {r}"
+    if axis == 0:
+        full = OC.all_reduce(bits, dtype="bf16", rounding="hop")
+        for r in range(t):
+            assert same_bits(host_bits(ar[r]), full[r]), f"AR replica {r}"
+
+
+def test_per_hop_and_end_rounding_differ_where_the_oracle_says():
+    # t = 3; chunk 0 sums U[1] = 1, U[2] = 2^-8, U[0] = 2^-8 in that order: one rounding at the end
+    # gives 1 + 2^-7 (0x3F81), rounding after every hop gives 1 (0x3F80), as the oracle's pins state.
+    t, rows, cols = 3, 3, 8
+    vals = {0: 0x3B80, 1: 0x3F80, 2: 0x3B80}
+    ins = []
+    for d in range(t):
+        b = np.zeros((rows, cols), dtype=np.uint16)
+        b[0, :] = vals[d]
+        ins.append(cuda(S.bits_to_bf16(b)))
+    outs = {}
+    for mode in (tp.TP_BF16, tp.TP_BF16_RING):
+        o = [torch.empty((rows // t, cols), dtype=torch.bfloat16, device="cuda") for _ in range(t)]
+        tp.tp_reduce_scatter(ins, o, rows, cols, 0, mode, t)
+        torch.cuda.synchronize()
+        outs[mode] = host_bits(o[0])
+    assert np.all(outs[tp.TP_BF16] == 0x3F81)
+    assert np.all(outs[tp.TP_BF16_RING] == 0x3F80)

@@ -61,6 +61,9 @@ CASES = [
     # odd k-block counts per shard on CTA pairs (two k-blocks per pipeline stage)
     (4, 1024, 768, 512, tp.TP_OUT_AR, 0),         # 192 per shard: three k-blocks
     (2, 512, 80, 512, tp.TP_OUT_RS, 0),           # 40 per shard: one ragged k-block
+    # axis 1 places no constraint on the row count: a partial last row-tile on the single-CTA kernel
+    (2, 200, 512, 512, tp.TP_OUT_RS, 1),
+    (4, 72, 256, 1024, tp.TP_OUT_RS, 1),
 ]
 
 

@@ -106,6 +106,16 @@ def test_mlp_shard_count_extremes(N, h, F, t, act):
         assert same_bits(rs[r], ar[0][r * N // t:(r + 1) * N // t]), f"RS block {r}"
 
 
+def tile_rows(n_rows: int, tile: int = 128) -> np.ndarray:
+    """One row from every `tile`-row block of the output, at an offset that moves across the block
+    from tile to tile (so different TMEM lanes, epilogue warps and both CTAs of a pair are checked),
+    plus the first and the last row."""
+    rows = {0, n_rows - 1}
+    for mt in range(n_rows // tile):
+        rows.add(mt * tile + (mt * 53 + 17) % tile)
+    return np.array(sorted(rows))
+
+
 # ---------------------------------------------------------------------------------- Llama-3-8B SwiGLU MLP
 @pytest.fixture(scope="module")
 def llama8b():
@@ -127,7 +137,9 @@ def test_llama8b_swiglu_mlp_sampled_rows(llama8b):
     # the reducing modes fuse the row GEMM with its collective: the partials come from PARTIALS mode
     _, partials, _ = _mlp_device(m["dX"], m["w_in"], m["w_down"], N, h, F, t, tp.TP_ACT_SWIGLU, tp.TP_OUT_PARTIALS)
     z, _, out = _mlp_device(m["dX"], m["w_in"], m["w_down"], N, h, F, t, tp.TP_ACT_SWIGLU, tp.TP_OUT_RS_AG)
-    rows = np.sort(np.random.default_rng(0).choice(N, 48, replace=False))
+    # every 128-row m-tile of the output (both GEMMs, every pair tile and the fused kernel's half-width
+    # last-round tiles: whole rows cover every n-tile)
+    rows = tile_rows(N)
     Xr = f64(m["X"])[rows]
     Wg = m["Wgu"][:, :F].float().numpy()
     Wu = m["Wgu"][:, F:].float().numpy()
@@ -192,9 +204,13 @@ def _run_case(case_id, strategy, xs, ws, B, D, F, t, c_dtype):
     return c, layout
 
 
+# Two shapes: with (512, 384, 768) case 2 AllGather materialises its gather (D/t = 96 is not whole
+# 64-wide k-blocks) while case 4 reads X's row pieces and W's column pieces in place; with
+# (384, 512, 640) it is the other way round (D/t = 128; B/t = 96, F/t = 160).
+@pytest.mark.parametrize("shape", [(512, 384, 768), (384, 512, 640)])
 @pytest.mark.parametrize("case_id,strategy", [(1, 0), (2, 0), (2, 1), (3, 0), (3, 1), (3, 2), (4, 0), (4, 1)])
-def test_cases_small_against_oracle(case_id, strategy):
-    B, D, F, t = 512, 384, 768, 4
+def test_cases_small_against_oracle(case_id, strategy, shape):
+    (B, D, F), t = shape, 4
     X, W = S.case_operands(seed=case_id, B=B, D=D, F=F)
     xs, ws = _case_shards(X, W, case_id, t)
     dxs = [cuda(x) for x in xs]
@@ -216,35 +232,67 @@ def test_cases_small_against_oracle(case_id, strategy):
             assert np.array_equal(host_bits(c16[i]), f32_to_bf16_bits(host_bits(c32[i])))
 
 
+@pytest.mark.parametrize("case_id,strategy", [(2, 0), (4, 0), (4, 1)])
+def test_gather_in_place_equals_gather_then_gemm(case_id, strategy):
+    """Reading the gathered operand's pieces where they lie gives the same bits as the AllGather into
+    a buffer followed by the plain grouped GEMM: the same MMA sequence runs on the same values."""
+    B, D, F, t = 1024, 512, 1536, 4
+    assert tp.tp_sharded_matmul_ws_bytes(case_id, strategy, B, D, F, t) == 0
+    X, W = S.case_operands(seed=40 + case_id + strategy, B=B, D=D, F=F)
+    xs, ws = _case_shards(X, W, case_id, t)
+    dxs = [cuda(x) for x in xs]
+    dws = [cuda(w) for w in ws]
+    c, _ = _run_case(case_id, strategy, dxs, dws, B, D, F, t, tp.TP_F32)
+    if case_id == 2:       # X gathered along D, every shard computes the full C
+        g = [torch.empty((B, D), dtype=torch.bfloat16, device="cuda") for _ in range(t)]
+        tp.tp_all_gather(dxs, g, B, D, 1, tp.TP_BF16, t)
+        ref = [torch.empty((B, F), device="cuda") for _ in range(t)]
+        tp.tp_grouped_gemm(t, g, dws, ref, B, F, D, tp.TP_ACT_NONE, tp.TP_F32)
+    elif strategy == 0:    # X gathered along B, shard i's columns of W
+        g = [torch.empty((B, D), dtype=torch.bfloat16, device="cuda") for _ in range(t)]
+        tp.tp_all_gather(dxs, g, B, D, 0, tp.TP_BF16, t)
+        ref = [torch.empty((B, F // t), device="cuda") for _ in range(t)]
+        tp.tp_grouped_gemm(t, g, dws, ref, B, F // t, D, tp.TP_ACT_NONE, tp.TP_F32)
+    else:                  # W gathered along F, shard i's rows of X
+        g = [torch.empty((D, F), dtype=torch.bfloat16, device="cuda") for _ in range(t)]
+        tp.tp_all_gather(dws, g, D, F, 1, tp.TP_BF16, t)
+        ref = [torch.empty((B // t, F), device="cuda") for _ in range(t)]
+        tp.tp_grouped_gemm(t, dxs, g, ref, B // t, F, D, tp.TP_ACT_NONE, tp.TP_F32)
+    torch.cuda.synchronize()
+    _status_ok()
+    for i in range(t):
+        assert torch.equal(c[i], ref[i]), f"shard {i}"
+
+
 @pytest.fixture(scope="module")
 def case_operands_full():
+    """The full-size case operands and the oracle's fp64 rows of the logical C = X W for one row of
+    every 128-row block (whole rows: all F columns), computed once for every strategy."""
     X, W = S.case_operands(seed=0)
-    return X, W
+    rows = tile_rows(X.shape[0])
+    ref = OM.matmul(f64(X[torch.from_numpy(rows)]), f64(W))
+    return X, W, rows, ref
 
 
 @pytest.mark.parametrize("case_id,strategy", [(1, 0), (2, 0), (2, 1), (3, 0), (3, 1), (3, 2), (4, 0), (4, 1)])
 def test_cases_full_size_sampled(case_operands_full, case_id, strategy):
     B, D, F, t = 8192, 8192, 28672, 4
-    X, W = case_operands_full
+    X, W, rows, ref = case_operands_full
     xs, ws = _case_shards(X, W, case_id, t)
     dxs = [cuda(x) for x in xs]
     dws = [cuda(w) for w in ws] if case_id != 1 and case_id != 2 else [cuda(W)] * t
     c, layout = _run_case(case_id, strategy, dxs, dws, B, D, F, t, tp.TP_F32)
-    g = np.random.default_rng(case_id * 10 + strategy)
-    rows = np.sort(g.choice(B, 24, replace=False))
-    cols = np.sort(g.choice(F, 96, replace=False))
-    ref = OM.matmul(f64(X[torch.from_numpy(rows)]), f64(W[:, torch.from_numpy(cols)]))
-    # gather the sampled logical entries from the shards
+    # whole logical rows, one from every 128-row m-tile of the output: every m-tile and n-tile of every
+    # shard's output is compared (replicated outputs: the row's replica rotates over the shards)
     got = np.empty_like(ref)
     for a, r in enumerate(rows):
-        for b, col in enumerate(cols):
-            if layout == "rows":
-                shard, rr, cc = r // (B // t), r % (B // t), col
-            elif layout == "cols":
-                shard, rr, cc = col // (F // t), r, col % (F // t)
-            else:
-                shard, rr, cc = (a + b) % t, r, col
-            got[a, b] = float(c[shard][rr, cc])
+        r = int(r)
+        if layout == "rows":
+            got[a] = f64(c[r // (B // t)][r % (B // t)])
+        elif layout == "cols":
+            got[a] = np.concatenate([f64(c[i][r]) for i in range(t)])
+        else:
+            got[a] = f64(c[a % t][r])
     assert_close(got, ref, GEMM_TOL, f"case {case_id} strategy {strategy}")
     if layout == "replicated":   # AllReduce: every replica bit-identical at full size
         for i in range(1, t):
@@ -277,7 +325,7 @@ def test_llama70b_layer_sampled_rows():
                     z_ws, partials, y)
     torch.cuda.synchronize()
     _status_ok()
-    rows = np.sort(np.random.default_rng(70).choice(N, 16, replace=False))
+    rows = tile_rows(N)   # every 128-row m-tile, whole rows (every n-tile)
     f32 = lambda x: x.float().numpy()  # noqa: E731  (exact widening of bf16)
     sh_qkv = OL.shard_qkv(f32(L["Wq"]), f32(L["Wk"]), f32(L["Wv"]), n_h, n_kv, d_h, t)
     sh_o = OL.shard_rows(f32(L["Wo"]), t)
