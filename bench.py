@@ -15,7 +15,9 @@ step per replica, summed over replicas / max-over-ranks time). Per-kernel CUDA-e
 timed region give the roofline of the dominant kernel (the column GEMM, tensor-bound); the standalone
 ReduceScatter loop gives the HBM roofline (algorithmic bytes (t+1)*M). `e2e` repeats the step through tp_mlp_fwd with
 X copied in from pinned host memory and the result copied back, every step. `cpu_baseline` times the
-oracle on a bounded row sample of the same workload on this host.
+oracle, single-threaded, on bounded row samples of the same workload on this host. On one GPU the line
+also carries `workloads`: the TP+SP forward, the 70B layer, every sharded-matmul strategy and ring
+collective points, each timed with CUDA events under one clock record.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 Multi-GPU: launched by torchrun, one process per GPU, each an independent replica (no collective
@@ -46,9 +48,8 @@ RS_BYTES = (T + 1) * M_PARTIAL                  # read t*M, write M
 AG_BYTES = T * M_PARTIAL                        # in place: read M once, write the t-1 other copies
 WORKLOAD = ("llama3-8b SwiGLU TP-MLP forward, t=8 virtual shards, 4096 tokens x h=4096, F=14336; "
             "column GEMM+SwiGLU -> row GEMM fused with ring ReduceScatter(tokens) + AllGather")
-CPU_SAMPLE_ROWS = 512
-REF_ROWS_PER_STEP = 64
-
+ORACLE_ROWS = 128          # token rows per oracle sample (the reference arm's step and cpu_baseline alike)
+CPU_BASELINE_SAMPLES = 8   # cpu_baseline: this many samples of ORACLE_ROWS rows each
 
 def _peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -184,7 +185,15 @@ def _oracle_step(Xs, shards_in, shards_down):
     return OC.all_gather(rs, axis=0)
 
 
+def _single_thread():
+    """Context that holds numpy's BLAS to one thread: the oracle is timed as the plain single-threaded
+    program it is meant to be, whatever BLAS the host's numpy links."""
+    from threadpoolctl import threadpool_limits
+    return threadpool_limits(limits=1, user_api="blas")
+
+
 def _blas_threads() -> int:
+    """Threads numpy's BLAS would use right now (1 inside _single_thread())."""
     try:
         from threadpoolctl import threadpool_info
         n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
@@ -193,41 +202,49 @@ def _blas_threads() -> int:
         return 1
 
 
-def cpu_baseline(rows: int = CPU_SAMPLE_ROWS) -> dict:
-    Xs, si, sd = _oracle_sample(rows)
-    t0 = time.perf_counter()
-    _oracle_step(Xs, si, sd)
-    dt = time.perf_counter() - t0
-    flops = FLOPS_STEP * rows / N_TOK
-    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": _blas_threads(), "kind": "oracle",
-            "sample": f"{rows} of {N_TOK} token rows of the same MLP (all 8 shards' fp64 GEMMs + fp32 ring RS/AG), "
-                      f"{dt:.2f} s; value = sample FLOPs / time"}
+def _oracle_rates(steps: int, warmup: int):
+    """Times the oracle on `steps` row samples of ORACLE_ROWS rows (after `warmup` untimed ones),
+    single-threaded. Returns (seconds per sample, BLAS threads used)."""
+    Xs_all, si, sd = _oracle_sample(ORACLE_ROWS * 4)
+    times = []
+    with _single_thread():
+        threads = _blas_threads()
+        for i in range(warmup + steps):
+            r0 = (i % 4) * ORACLE_ROWS
+            t0 = time.perf_counter()
+            _oracle_step(Xs_all[r0:r0 + ORACLE_ROWS], si, sd)
+            if i >= warmup:
+                times.append(time.perf_counter() - t0)
+    return sum(times) / len(times), threads
+
+
+def _oracle_sample_text(n: int, per: float) -> str:
+    return (f"{n} samples of {ORACLE_ROWS} of {N_TOK} token rows of the same MLP (all 8 shards' fp64 GEMMs + "
+            f"binary32 ring RS/AG), {per:.2f} s each, single-threaded; value = sample FLOPs / time")
+
+
+def cpu_baseline() -> dict:
+    per, threads = _oracle_rates(CPU_BASELINE_SAMPLES, 1)
+    flops = FLOPS_STEP * ORACLE_ROWS / N_TOK
+    return {"value": flops / per / 1e12, "unit": "TFLOP/s", "cores": threads, "host_cpus": os.cpu_count(),
+            "blas_threads": threads, "kind": "oracle", "sample": _oracle_sample_text(CPU_BASELINE_SAMPLES, per)}
 
 
 def run_reference(args) -> int:
     ws, rank, _ = _dist_env()
     if rank != 0:
         return 0
-    Xs_all, si, sd = _oracle_sample(REF_ROWS_PER_STEP * 4)
-    times = []
-    for i in range(args.warmup + args.steps):
-        r0 = (i % 4) * REF_ROWS_PER_STEP
-        Xs = Xs_all[r0:r0 + REF_ROWS_PER_STEP]
-        t0 = time.perf_counter()
-        _oracle_step(Xs, si, sd)
-        if i >= args.warmup:
-            times.append(time.perf_counter() - t0)
-    per_step = sum(times) / len(times)
-    flops = FLOPS_STEP * REF_ROWS_PER_STEP / N_TOK
+    per_step, threads = _oracle_rates(args.steps, args.warmup)
+    flops = FLOPS_STEP * ORACLE_ROWS / N_TOK
     value = flops / per_step / 1e12
-    cores = _blas_threads()
     _emit({
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "sample_rows_per_step": REF_ROWS_PER_STEP},
-        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                         "sample": f"{REF_ROWS_PER_STEP} of {N_TOK} token rows per step"},
+        "config": {"workload": WORKLOAD, "sample_rows_per_step": ORACLE_ROWS},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "host_cpus": os.cpu_count(),
+                         "blas_threads": threads, "kind": "oracle",
+                         "sample": _oracle_sample_text(args.steps, per_step)},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     })
     return 0
@@ -391,6 +408,13 @@ def run_gpu(args) -> int:
     torch.cuda.synchronize()
     d2h_gbs = d_iters * N_TOK * H * 4 / (d_start.elapsed_time(d_stop) * 1e-3) / 1e9
 
+    # ---- the other workloads (one GPU only: the scaling runs time the headline step alone) ---------
+    extra = None
+    if ws == 1 and not args.no_workloads:
+        del outs, x_dev, y_host, x_host
+        torch.cuda.empty_cache()
+        extra = workloads(X, w_in, w_down, z)
+
     # ---- max over ranks ------------------------------------------------------------------------
     total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dist, dev)
     n = ws
@@ -444,6 +468,8 @@ def run_gpu(args) -> int:
             "gpu_launches": 2 * args.steps,
             "clocks": clk,
         }
+        if extra is not None:
+            line["workloads"] = extra
         if not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline()
         _emit(line)
@@ -469,67 +495,66 @@ def _time_ms(fn, iters: int, warmup: int = 3) -> float:
     return a.elapsed_time(b) / iters
 
 
-def run_sweep(args) -> int:
-    """The collective sweep: ReduceScatter, AllGather and AllReduce in ring order over t in {2,4,8} shard
-    buffers, fp32 and bf16, payload M = 1 MiB .. 1 GiB in powers of 4 (M = each shard's full buffer for
-    RS/AR, the gathered tensor for AG). GB/s = algorithmic bytes / time: RS and AG (t+1)M, AR 2tM."""
+def _iters_for(expected_ms: float, budget_ms: float = 60.0, lo: int = 5, hi: int = 200) -> int:
+    return max(lo, min(hi, int(budget_ms / max(expected_ms, 1e-3))))
+
+
+def collective_point(t: int, dt: str, mib: int, op: str) -> dict:
+    """One point of the collective sweep: ReduceScatter / AllGather / AllReduce in ring order over t
+    shard buffers resident in HBM. M = each shard's full buffer for RS/AR, the gathered tensor for AG.
+    GB/s = algorithmic bytes / time: RS and AG (t+1)M, AR 2tM; ring_bus_gbs is the NCCL-style
+    (t-1)/t M (x2 for AR) over the same time."""
     import torch
     import tensor_sharded_matmul_b200 as tp
-    hbm_peak = _peaks()[0]
-    torch.cuda.set_device(0)
-    for t in (2, 4, 8):
-        for dt in ("f32", "bf16"):
-            es = 4 if dt == "f32" else 2
-            tdt = torch.float32 if dt == "f32" else torch.bfloat16
-            for mib in (1, 4, 16, 64, 256, 1024):
-                elems = mib * (1 << 20) // es
-                cols = 4096 if elems >= 4096 * 64 else 256
-                rows = elems // cols
-                for op in ("RS", "AG", "AR"):
-                    if op == "AG":
-                        ins = [torch.empty((rows // t, cols), dtype=tdt, device="cuda").normal_() for _ in range(t)]
-                        outs = [torch.empty((rows, cols), dtype=tdt, device="cuda") for _ in range(t)]
-                        fn = lambda: tp.tp_all_gather(ins, outs, rows, cols, 0, tp.TP_F32 if dt == "f32" else tp.TP_BF16, t)  # noqa: E731
-                        nbytes = (t + 1) * mib * (1 << 20)
-                    else:
-                        ins = [torch.empty((rows, cols), dtype=tdt, device="cuda").normal_() for _ in range(t)]
-                        shape = (rows // t, cols) if op == "RS" else (rows, cols)
-                        outs = [torch.empty(shape, dtype=tdt, device="cuda") for _ in range(t)]
-                        code = tp.TP_F32 if dt == "f32" else tp.TP_BF16
-                        if op == "RS":
-                            fn = lambda: tp.tp_reduce_scatter(ins, outs, rows, cols, 0, code, t)  # noqa: E731
-                            nbytes = (t + 1) * mib * (1 << 20)
-                        else:
-                            fn = lambda: tp.tp_all_reduce(ins, outs, rows, cols, code, t)  # noqa: E731
-                            nbytes = 2 * t * mib * (1 << 20)
-                    iters = max(5, min(200, int(2e9 / nbytes)))
-                    ms = _time_ms(fn, iters)
-                    gbs = nbytes / (ms * 1e-3) / 1e9
-                    bus = (t - 1) / t * mib * (1 << 20) * (2 if op == "AR" else 1) / (ms * 1e-3) / 1e9
-                    _emit({"config": "collective_sweep", "op": op, "t": t, "dtype": dt, "payload_mib": mib,
-                           "ms": ms, "gbs": gbs, "frac_hbm": gbs / hbm_peak, "ring_bus_gbs": bus})
-                    del ins, outs
-                    torch.cuda.empty_cache()
-    return 0
+    es = 4 if dt == "f32" else 2
+    tdt = torch.float32 if dt == "f32" else torch.bfloat16
+    code = tp.TP_F32 if dt == "f32" else tp.TP_BF16
+    elems = mib * (1 << 20) // es
+    cols = 4096 if elems >= 4096 * 64 else 256
+    rows = elems // cols
+    if op == "AG":
+        ins = [torch.empty((rows // t, cols), dtype=tdt, device="cuda").normal_() for _ in range(t)]
+        outs = [torch.empty((rows, cols), dtype=tdt, device="cuda") for _ in range(t)]
+        fn = lambda: tp.tp_all_gather(ins, outs, rows, cols, 0, code, t)  # noqa: E731
+        nbytes = (t + 1) * mib * (1 << 20)
+    else:
+        ins = [torch.empty((rows, cols), dtype=tdt, device="cuda").normal_() for _ in range(t)]
+        shape = (rows // t, cols) if op == "RS" else (rows, cols)
+        outs = [torch.empty(shape, dtype=tdt, device="cuda") for _ in range(t)]
+        if op == "RS":
+            fn = lambda: tp.tp_reduce_scatter(ins, outs, rows, cols, 0, code, t)  # noqa: E731
+            nbytes = (t + 1) * mib * (1 << 20)
+        else:
+            fn = lambda: tp.tp_all_reduce(ins, outs, rows, cols, code, t)  # noqa: E731
+            nbytes = 2 * t * mib * (1 << 20)
+    ms = _time_ms(fn, _iters_for(nbytes / 6.0e9, 200.0))
+    del ins, outs
+    torch.cuda.empty_cache()
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    bus = (t - 1) / t * mib * (1 << 20) * (2 if op == "AR" else 1) / (ms * 1e-3) / 1e9
+    return {"ms": ms, "gbs": gbs, "frac_hbm": gbs / _peaks()[0], "ring_bus_gbs": bus, "bytes": nbytes}
 
 
-def run_cases(args) -> int:
-    """The four sharded-matmul cases of C[B,F] = X[B,D] W[D,F] at B=D=8192, F=28672 over t=4 shards,
-    every strategy; TFLOP/s counts the FLOPs executed (case 2 AllGather computes C on every shard)."""
+CASE_NAMES = {(1, 0): "local", (2, 0): "allgather", (2, 1): "allreduce", (3, 0): "allreduce", (3, 1): "rs_b",
+              (3, 2): "rs_f", (4, 0): "gather_x", (4, 1): "gather_w"}
+
+
+def sharded_matmul_cases(which=None):
+    """The four sharded-matmul cases of C[B,F] = X[B,D] W[D,F] at B=D=8192, F=28672 over t=4 shards
+    (`which`: the (case, strategy) pairs to time, default all). TFLOP/s counts the FLOPs executed
+    (case 2 AllGather computes C on every shard). Yields (case, strategy, name, ms, tflops, ws_bytes)."""
     import torch
     import synthetic as S
     import tensor_sharded_matmul_b200 as tp
-    torch.cuda.set_device(0)
     B, D, F, t = 8192, 8192, 28672, 4
     X, W = S.case_operands(seed=0, device="cuda")
-    peak = _peaks()[1]
     shard = {1: (list(X.chunk(t, 0)), [W] * t), 2: (list(X.chunk(t, 1)), [W] * t),
              3: (list(X.chunk(t, 1)), list(W.chunk(t, 0))), 4: (list(X.chunk(t, 0)), list(W.chunk(t, 1)))}
-    names = {(1, 0): "local", (2, 0): "allgather", (2, 1): "allreduce", (3, 0): "allreduce", (3, 1): "rs_b",
-             (3, 2): "rs_f", (4, 0): "gather_x", (4, 1): "gather_w"}
     shapes = {(1, 0): (B // t, F), (2, 0): (B, F), (2, 1): (B, F), (3, 0): (B, F), (3, 1): (B // t, F),
               (3, 2): (B, F // t), (4, 0): (B, F // t), (4, 1): (B // t, F)}
-    for (case_id, strategy), name in names.items():
+    for (case_id, strategy), name in CASE_NAMES.items():
+        if which is not None and (case_id, strategy) not in which:
+            continue
         xs, ws = shard[case_id]
         xs = [x.contiguous() for x in xs]
         ws = [w.contiguous() for w in ws] if case_id in (3, 4) else ws
@@ -537,22 +562,19 @@ def run_cases(args) -> int:
         nbytes = tp.tp_sharded_matmul_ws_bytes(case_id, strategy, B, D, F, t)
         wsb = torch.empty(max(nbytes, 256), dtype=torch.uint8, device="cuda")
         fn = lambda: tp.tp_sharded_matmul(case_id, strategy, xs, ws, B, D, F, t, c, tp.TP_F32, wsb, nbytes)  # noqa: E731
-        ms = _time_ms(fn, 10)
         flops = 2.0 * B * D * F * (t if (case_id, strategy) == (2, 0) else 1)
-        _emit({"config": "sharded_matmul", "case": case_id, "strategy": name, "ms": ms,
-               "tflops_executed": flops / (ms * 1e-3) / 1e12, "frac_bf16_peak": flops / (ms * 1e-3) / 1e12 / peak})
+        ms = _time_ms(fn, _iters_for(flops / 1.2e12, 60.0, lo=5, hi=50))
+        yield case_id, strategy, name, ms, flops / (ms * 1e-3) / 1e12, nbytes
         del c, wsb, xs, ws
         torch.cuda.empty_cache()
-    return 0
 
 
-def run_layer70b(args) -> int:
+def layer70b():
     """One Llama-3-70B-shaped TP=8 layer on 2048 tokens without its attention core (QKV column GEMM,
-    W_O row GEMM + AllReduce + residual, SwiGLU MLP + AllReduce + residual)."""
+    W_O row GEMM + AllReduce + residual, SwiGLU MLP + AllReduce + residual). Returns (ms, GFLOP)."""
     import torch
     import synthetic as S
     import tensor_sharded_matmul_b200 as tp
-    torch.cuda.set_device(0)
     N, h, n_h, n_kv, d_h, F, t = 2048, 8192, 64, 8, 128, 28672, 8
     L = S.llama70b_layer(seed=0, device="cuda")
     qkv_w = (n_h // t + 2 * (n_kv // t)) * d_h
@@ -574,10 +596,133 @@ def run_layer70b(args) -> int:
     y = [torch.empty((N, h), device="cuda") for _ in range(t)]
     fn = lambda: tp.tp_layer_fwd(X, o, N, h, n_h, n_kv, d_h, F, t, w_qkv, w_o, w_gu, w_down, qkv, h1, h1b, z,  # noqa: E731
                                  None, y)
-    ms = _time_ms(fn, 50)
     flops = 2.0 * N * (h * qkv_w * t + n_h * d_h * h + h * 2 * F + F * h)
-    _emit({"config": "llama70b_tp8_layer", "tokens": N, "ms": ms, "gflop": flops / 1e9,
-           "tflops": flops / (ms * 1e-3) / 1e12, "frac_bf16_peak": flops / (ms * 1e-3) / 1e12 / _peaks()[1]})
+    ms = _time_ms(fn, 30)
+    del w_qkv, w_o, w_gu, w_down, o, X, qkv, h1, h1b, z, y
+    torch.cuda.empty_cache()
+    return ms, flops / 1e9
+
+
+def workloads(X, w_in, w_down, z) -> dict:
+    """The other workloads, each timed with CUDA events on the current stream after warm-up, under one
+    nvidia-smi clock record: the 70B layer, every sharded-matmul strategy, the TP+SP MLP forward on the
+    8B shape (reusing the headline step's weights) and the ring collectives at t in {2, 8}, fp32/bf16,
+    64 MiB and 1 GiB. Fractions are of the measured burst peaks (each kernel is timed in a short loop)."""
+    import torch
+    import tensor_sharded_matmul_b200 as tp
+    hbm, burst, _, src = _peaks()
+    out = {"peak_source": f"{src} (bf16 burst, hbm copy)"}
+    clocks = ClockSampler(None)
+    clocks.start()
+    time.sleep(0.2)
+    t0 = time.perf_counter()
+    # the TP + SP MLP forward (AllGather along tokens fused into the column GEMM's operand loads,
+    # ReduceScatter fused into the row GEMM), on the headline step's weights
+    t, N, h = T, N_TOK, H
+    x_shards = [X[r * N // t:(r + 1) * N // t].contiguous() for r in range(t)]
+    out_sp = [torch.empty((N // t, h), device="cuda") for _ in range(t)]
+    ms = _time_ms(lambda: tp.tp_mlp_fwd_sp(x_shards, N, h, F, t, tp.TP_ACT_SWIGLU, w_in, w_down, z, out_sp), 50)
+    rate = FLOPS_STEP / (ms * 1e-3) / 1e12
+    out["tp_sp_mlp_fwd_llama8b"] = {"ms": ms, "tflops": rate, "frac_bf16_peak": rate / burst}
+    del x_shards, out_sp
+    ms, gflop = layer70b()
+    rate = gflop / ms
+    out["llama70b_tp8_layer"] = {"ms": ms, "tflops": rate, "frac_bf16_peak": rate / burst, "gflop": gflop}
+    for case_id, strategy, name, ms, rate, nbytes in sharded_matmul_cases():
+        out[f"case{case_id}_{name}"] = {"ms": ms, "tflops": rate, "frac_bf16_peak": rate / burst,
+                                        "workspace_bytes": nbytes}
+    coll = {}
+    for t_ in (2, 8):
+        for dt in ("f32", "bf16"):
+            for mib in (64, 1024):
+                for op in ("RS", "AG", "AR"):
+                    r = collective_point(t_, dt, mib, op)
+                    coll[f"{op}_t{t_}_{dt}_{mib}MiB"] = {k: r[k] for k in ("ms", "gbs", "frac_hbm")}
+    out["collectives"] = coll
+    out["wall_s"] = time.perf_counter() - t0
+    out["clocks"] = clocks.stop()
+    st, site = tp.tp_device_status(1)
+    if st != tp.TP_OK:
+        raise RuntimeError(f"device wait ran out at site {site}")
+    return out
+
+
+def run_sweep(args) -> int:
+    """The collective sweep: ReduceScatter, AllGather and AllReduce in ring order over t in {2,4,8} shard
+    buffers, fp32 and bf16, payload M = 1 MiB .. 1 GiB in powers of 4 (M = each shard's full buffer for
+    RS/AR, the gathered tensor for AG). GB/s = algorithmic bytes / time: RS and AG (t+1)M, AR 2tM."""
+    import torch
+    torch.cuda.set_device(0)
+    for t in (2, 4, 8):
+        for dt in ("f32", "bf16"):
+            for mib in (1, 4, 16, 64, 256, 1024):
+                for op in ("RS", "AG", "AR"):
+                    r = collective_point(t, dt, mib, op)
+                    _emit({"config": "collective_sweep", "op": op, "t": t, "dtype": dt, "payload_mib": mib,
+                           **{k: r[k] for k in ("ms", "gbs", "frac_hbm", "ring_bus_gbs")}})
+    return 0
+
+
+def run_cases(args) -> int:
+    """The four sharded-matmul cases at B=D=8192, F=28672 over t=4 shards, every strategy."""
+    import torch
+    torch.cuda.set_device(0)
+    peak = _peaks()[1]
+    for case_id, strategy, name, ms, rate, nbytes in sharded_matmul_cases():
+        _emit({"config": "sharded_matmul", "case": case_id, "strategy": name, "ms": ms, "tflops_executed": rate,
+               "frac_bf16_peak": rate / peak, "workspace_bytes": nbytes})
+    return 0
+
+
+def run_layer70b(args) -> int:
+    """One Llama-3-70B-shaped TP=8 layer on 2048 tokens without its attention core."""
+    import torch
+    torch.cuda.set_device(0)
+    ms, gflop = layer70b()
+    _emit({"config": "llama70b_tp8_layer", "tokens": 2048, "ms": ms, "gflop": gflop,
+           "tflops": gflop / ms, "frac_bf16_peak": gflop / ms / _peaks()[1]})
+    return 0
+
+
+ROW_REDUCE_SHAPES = {
+    # name: (t, tokens, k (the full contraction), n, reduce mode) of tp_row_linear_reduce
+    "8b_rs_ag": (8, 4096, 14336, 4096, "RS_AG"),     # Llama-3-8B down projection, RS along tokens + AG
+    "8b_rs": (8, 4096, 14336, 4096, "RS"),           # the same, ReduceScatter only (TP+SP exit)
+    "70b_wo_ar": (8, 2048, 8192, 8192, "AR"),        # Llama-3-70B attention output projection + AR
+    "70b_down_ar": (8, 2048, 28672, 8192, "AR"),     # Llama-3-70B down projection + AR
+}
+
+
+def run_rowreduce(args) -> int:
+    """The row-parallel GEMM fused with its ring collective (tp_row_linear_reduce) on the Llama-3 8B
+    and 70B shapes, one JSON line per shape: x bf16 [t][N][k/t] ~N(0,1), w bf16 [t][k/t][n] ~N(0,0.02).
+    TFLOP/s counts 2*N*k*n; the fraction is of the measured bf16 burst peak."""
+    import torch
+    import synthetic as S
+    import tensor_sharded_matmul_b200 as tp
+    torch.cuda.set_device(0)
+    burst = _peaks()[1]
+    modes = {"RS": tp.TP_OUT_RS, "AR": tp.TP_OUT_AR, "RS_AG": tp.TP_OUT_RS_AG}
+    names = [args.shape] if args.shape else list(ROW_REDUCE_SHAPES)
+    for name in names:
+        t, N, k, n, mode = ROW_REDUCE_SHAPES[name]
+        d = S.Draw(7, "cuda")
+        x = d.normal((t, N, k // t), 1.0)
+        w = d.normal((t, k // t, n), 0.02)
+        rows = N // t if mode == "RS" else N
+        out = [torch.empty((rows, n), device="cuda") for _ in range(t)]
+        fn = lambda: tp.tp_row_linear_reduce(x, N, k, n, t, w, modes[mode], 0, out)  # noqa: E731
+        ms = _time_ms(fn, args.steps if args.steps < 500 else 50)
+        rate = 2.0 * N * k * n / (ms * 1e-3) / 1e12
+        _emit({"config": "rowreduce", "shape": name, "t": t, "tokens": N, "k": k, "n": n, "mode": mode, "ms": ms,
+               "tflops": rate, "frac_bf16_peak": rate / burst,
+               "bytes_written": t * rows * n * 4})
+        del x, w, out
+        torch.cuda.empty_cache()
+    st, site = tp.tp_device_status(1)
+    if st != tp.TP_OK:
+        print(f"device wait ran out at site {site}", file=sys.stderr)
+        return 3
     return 0
 
 
@@ -654,8 +799,12 @@ def main(argv=None) -> int:
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (profiling runs)")
-    ap.add_argument("--config", choices=["mlp8b", "sweep", "cases", "layer70b", "next"], default="mlp8b",
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="time the headline step only (profiling runs; multi-GPU runs always do)")
+    ap.add_argument("--config", choices=["mlp8b", "sweep", "cases", "layer70b", "next", "rowreduce"], default="mlp8b",
                     help="mlp8b: the headline step (one JSON line); the others print one line per measurement")
+    ap.add_argument("--shape", choices=sorted(ROW_REDUCE_SHAPES), default=None,
+                    help="--config rowreduce: one shape only (default: all)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
@@ -669,6 +818,8 @@ def main(argv=None) -> int:
         return run_layer70b(args)
     if args.config == "next":
         return run_next(args)
+    if args.config == "rowreduce":
+        return run_rowreduce(args)
     return run_gpu(args)
 
 
