@@ -172,12 +172,14 @@ def all_gather(bufs, axis: int = 0):
     return [np.concatenate([hold[i][k] for k in range(t)], axis=axis) for i in range(t)]
 
 
-def all_reduce(bufs, dtype: str = "f32", out_dtype: str | None = None, rounding: str = "end"):
-    """AllReduce = ReduceScatter (along rows) followed by AllGather: every shard ends with the full
-    ring-ordered sum. With bf16 the one rounding happens at the end of the ReduceScatter (or after
-    every hop, with rounding="hop")."""
-    rs = reduce_scatter(bufs, axis=0, dtype=dtype, out_dtype=out_dtype, rounding=rounding)
-    return all_gather(rs, axis=0)
+def all_reduce(bufs, dtype: str = "f32", out_dtype: str | None = None, rounding: str = "end", axis: int = 0):
+    """AllReduce = ReduceScatter followed by AllGather along the same axis: every shard ends with the
+    full ring-ordered sum. The ReduceScatter may scatter along either dimension ("Scaling Book 入门第 6
+    章", §6.4), which decides each element's summation order: rows (axis 0, the default) or columns
+    (axis 1). With bf16 the one rounding happens at the end of the ReduceScatter (or after every hop,
+    with rounding="hop")."""
+    rs = reduce_scatter(bufs, axis=axis, dtype=dtype, out_dtype=out_dtype, rounding=rounding)
+    return all_gather(rs, axis=axis)
 
 
 def all_to_all(bufs, split_axis: int, concat_axis: int):

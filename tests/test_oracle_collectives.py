@@ -270,3 +270,22 @@ def test_per_hop_bf16_equals_sequential_bf16_adds(t):
 def test_per_hop_mode_is_bf16_only():
     with pytest.raises(ValueError):
         C.reduce_scatter([np.zeros((2, 2), np.float32)] * 2, dtype="f32", rounding="hop")
+
+
+@pytest.mark.parametrize("t,axis", [(2, 1), (3, 1), (4, 0), (4, 1)])
+def test_all_reduce_along_either_axis_brute_force(t, axis):
+    # AllReduce = ReduceScatter + AllGather along one axis: element (r, c) of every replica is the
+    # ring sum of the chunk that holds it (rows for axis 0, columns for axis 1), added one binary32
+    # add at a time starting at shard chunk+1 -- checked element by element by brute force.
+    g = np.random.default_rng(60 + 10 * t + axis)
+    rows, cols = 3 * t, 2 * t
+    bufs = [(g.standard_normal((rows, cols)) * np.exp(g.standard_normal((rows, cols)) * 3)).astype(np.float32)
+            for _ in range(t)]
+    got = C.all_reduce(bufs, axis=axis)
+    ref = np.concatenate(_elementwise_ring_sum(bufs, t, axis), axis=axis)
+    for r in range(t):
+        assert np.array_equal(got[r].view(np.uint32), ref.view(np.uint32))
+    # the two axes order the adds differently (visible in binary32 on this data)
+    if t >= 3:
+        other = C.all_reduce(bufs, axis=1 - axis)
+        assert not np.array_equal(got[0].view(np.uint32), other[0].view(np.uint32))
