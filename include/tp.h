@@ -192,9 +192,13 @@ tp_status tp_row_linear(const uint16_t* x, int64_t N, int64_t k, int64_t n, int 
  * shard products in ring order (c+1, ..., c for the tile's chunk c), accumulates them in binary32
  * exactly as tp_reduce_scatter would, and writes the tile once:
  *   TP_OUT_RS           out[r] receives chunk r: [N/t, n] (axis 0) or [N, n/t] (axis 1)
- *   TP_OUT_AR, RS_AG    every out[r] receives the whole [N, n] sum (ReduceScatter with its AllGather
- *                       folded into the same epilogue; bit-identical to tp_all_reduce)
- * Results are bit-identical to tp_row_linear followed by tp_reduce_scatter / tp_all_reduce.
+ *   TP_OUT_AR           every out[r] receives the whole [N, n] sum: a ReduceScatter along `axis`
+ *                       (which fixes each element's summation order: its row chunk for 0, its
+ *                       column chunk for 1; [CH06] §6.4) with its AllGather folded into the same
+ *                       epilogue
+ *   TP_OUT_RS_AG        as TP_OUT_AR with the ReduceScatter along tokens (axis 0), whatever `axis` says
+ * Results are bit-identical to tp_row_linear followed by tp_reduce_scatter(axis) (and, for the
+ * AllReduce modes, tp_all_gather(axis); for axis 0 that is tp_all_reduce).
  * The fused kernel needs (N/t) % 128 == 0 for axis 0, or (n/t) % 256 == 0 for axis 1. Otherwise
  * `partials` (t fp32 [N, n] buffers, else NULL) is used for the unfused path, and without it the
  * call returns TP_EUNSUPPORTED. Aligned; k/t and n multiples of 8. */
@@ -290,8 +294,12 @@ tp_status tp_sharded_matmul(int case_id, int strategy, const uint16_t* const* x,
  *   qkv_out bf16 stacked [t][N][(n_h/t + 2kv)*d_h]
  *   h1     t fp32 [N, h] (replicas of the residual stream after attention); h1_bf16 bf16 [N, h]
  *   z_ws   bf16 [t][N][F/t]; y t fp32 [N, h]
- *   partials t fp32 [N, h] scratch, needed only when (N/t) % 128 != 0; otherwise both row GEMMs are
- *          fused with their AllReduce (and residual) and partials may be NULL
+ *   partials t fp32 [N, h] scratch, needed only when neither (h/t) % 256 == 0 nor (N/t) % 128 == 0;
+ *          otherwise both row GEMMs are fused with their AllReduce (and residual) and partials may
+ *          be NULL
+ * Both AllReduces scatter along h (their summation order follows column chunks of h/t) when
+ * (h/t) % 256 == 0, else along tokens: along h, all row-tiles of a chunk read the same shard's weight
+ * panel at the same time, so the weights stream from DRAM about once rather than once per row-tile.
  * ------------------------------------------------------------------------------------------------ */
 tp_status tp_layer_fwd(const uint16_t* x, const uint16_t* const* o, int64_t N, int64_t h, int n_h, int n_kv,
                        int d_h, int64_t F, int t, const uint16_t* w_qkv, const uint16_t* w_o,

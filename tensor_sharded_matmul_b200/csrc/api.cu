@@ -173,7 +173,7 @@ tp_status tp_row_linear_reduce(const uint16_t* x, int64_t N, int64_t k, int64_t 
   if (x == nullptr || w == nullptr || out == nullptr) return fail(TP_EINVAL, "null pointer");
   if (mode != TP_OUT_RS && mode != TP_OUT_AR && mode != TP_OUT_RS_AG) return fail(TP_EINVAL, "mode must reduce");
   if (axis != 0 && axis != 1) return fail(TP_EINVAL, "axis must be 0 or 1");
-  if (mode != TP_OUT_RS) axis = 0;
+  if (mode == TP_OUT_RS_AG) axis = 0;   // ReduceScatter along tokens, by definition
   if (k % t) return fail(TP_EDIVIS, "t=%d does not divide k=%lld", t, (long long)k);
   if (axis == 0 ? N % t != 0 : n % t != 0) return fail(TP_EDIVIS, "t=%d does not divide the scattered dim", t);
   if (ring_gemm_fits(N, n, t, axis))
@@ -415,20 +415,26 @@ tp_status tp_layer_fwd(const uint16_t* x, const uint16_t* const* o, int64_t N, i
   const int64_t kv = t <= n_kv ? n_kv / t : 1;
   const int64_t qkv_w = (n_h / t + 2 * kv) * d_h;
   const int64_t o_w = int64_t(n_h) * d_h / t;
-  const bool need_partials = !ring_gemm_fits(N, h, t, 0);
+  // Both AllReduces are fused into their row GEMMs. Their ReduceScatter scatters along h (columns)
+  // when h/t is a whole number of 256-column tiles: every row-tile of a chunk then reads the same
+  // shard's weight panel at the same time, so the weights stream from DRAM about once instead of once
+  // per row-tile. Otherwise along tokens (rows), else unfused through the partials.
+  const int ar_axis = ring_gemm_fits(N, h, t, 1) ? 1 : 0;
+  const bool need_partials = !ring_gemm_fits(N, h, t, ar_axis);
   if (need_partials && partials == nullptr) return fail(TP_EINVAL, "null partials (needed: N/t is not a multiple of 128)");
   for (int r = 0; r < t; ++r)
     if (o[r] == nullptr || h1[r] == nullptr || y[r] == nullptr || (need_partials && partials[r] == nullptr))
       return fail(TP_EINVAL, "null shard buffer %d", r);
   // 1. fused QKV projection, column-parallel on head boundaries (feeds the attention core)
   if (tp_status st = column_gemm(x, N, h, qkv_w, t, TP_ACT_NONE, w_qkv, qkv_out, s)) return st;
-  const bool fused = ring_gemm_fits(N, h, t, 0);
+  const bool fused = !need_partials;
   // 2-3. attention output projection (row-parallel) and g: AllReduce, with the residual add
   //      h1 = X + attn and the bf16 copy for the MLP input
   if (fused) {
     RingGemmArgs rg;
     std::memset(&rg, 0, sizeof(rg));
     rg.t = t; rg.M = N; rg.N = h; rg.K = o_w; rg.lda = o_w; rg.ldb = h; rg.op = RING_AR; rg.out_dtype = TP_F32;
+    rg.axis = ar_axis;
     rg.resid = x; rg.resid_dtype = TP_BF16; rg.copy_bf16 = h1_bf16;
     for (int r = 0; r < t; ++r) { rg.a[r] = o[r]; rg.b[r] = w_o + r * o_w * h; rg.out[r] = h1[r]; }
     if (tp_status st = ring_gemm(rg, s)) return st;
@@ -441,7 +447,7 @@ tp_status tp_layer_fwd(const uint16_t* x, const uint16_t* const* o, int64_t N, i
   // 4. SwiGLU MLP on bf16(h1), then AllReduce with y = h1 + mlp
   const int64_t f = F / t;
   if (tp_status st = column_gemm(h1_bf16, N, h, f, t, TP_ACT_SWIGLU, w_gu, z_ws, s)) return st;
-  if (fused) return fused_row_reduce(z_ws, N, f, h, t, w_down, TP_OUT_AR, 0, y, h1[0], TP_F32, nullptr, s);
+  if (fused) return fused_row_reduce(z_ws, N, f, h, t, w_down, TP_OUT_AR, ar_axis, y, h1[0], TP_F32, nullptr, s);
   if (tp_status st = row_gemm(z_ws, N, f, h, t, w_down, partials, s)) return st;
   return reduce_partials(partials, N, h, t, TP_OUT_AR, y, h1[0], TP_F32, nullptr, s);
 }

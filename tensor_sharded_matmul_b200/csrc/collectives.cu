@@ -126,6 +126,21 @@ struct IO<uint16_t, 1> {
   }
 };
 
+// Widening of one raw 16-byte vector of the input type (4 fp32 or 8 bf16 values) to binary32.
+template <typename T, int VEC>
+__device__ __forceinline__ void unpack16(const uint4& r, float (&f)[VEC]) {
+  if constexpr (sizeof(T) == 4) {
+    f[0] = __uint_as_float(r.x); f[1] = __uint_as_float(r.y); f[2] = __uint_as_float(r.z); f[3] = __uint_as_float(r.w);
+  } else {
+    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      f[2 * k] = __uint_as_float(w[k] << 16);
+      f[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+    }
+  }
+}
+
 // Chunk of full-tensor element e, and e's offset inside that chunk's shard buffer.
 __device__ __forceinline__ void locate(const RingParams& p, int64_t e, int& c, int64_t& local) {
   if (p.axis == 0) {
@@ -143,7 +158,8 @@ __device__ __forceinline__ void locate(const RingParams& p, int64_t e, int& c, i
 // residual (if any) and writes every replica (and the bf16 copy); ReduceScatter writes shard c's
 // piece.
 template <typename Tout, int VEC, bool AR>
-__device__ __forceinline__ void finish_unit(const RingParams& p, int64_t e, int c, float (&acc)[VEC], int t) {
+__device__ __forceinline__ void finish_unit(const RingParams& p, int64_t e, int c, int64_t local, float (&acc)[VEC],
+                                            int t) {
   if constexpr (AR) {
     if (p.resid != nullptr) {
       float r[VEC];
@@ -157,9 +173,6 @@ __device__ __forceinline__ void finish_unit(const RingParams& p, int64_t e, int 
     for (int s = 0; s < t; ++s) IO<Tout, VEC>::store(p.out[s], e, acc);
     if (p.copy_bf16 != nullptr) IO<uint16_t, VEC>::store(p.copy_bf16, e, acc);
   } else {
-    int cc;
-    int64_t local;
-    locate(p, e, cc, local);
     IO<Tout, VEC>::store(p.out[c], local, acc);
   }
 }
@@ -180,17 +193,19 @@ __global__ void __launch_bounds__(256) ring_reduce_kernel(const __grid_constant_
   const int64_t units = p.rows * p.cols / VEC;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t u0 = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; u0 < units; u0 += UNR * stride) {
-    if constexpr (TT > 0) {
-      float v[UNR][TT][VEC];
+    if constexpr (TT > 0 && VEC * sizeof(Tin) == 16) {
+      // raw 16-byte vectors: every load of the step is issued before any value is widened or added
+      uint4 raw[UNR][TT];
       int cs[UNR];
+      int64_t locs[UNR];
 #pragma unroll
       for (int k = 0; k < UNR; ++k) {
         const int64_t u = u0 + k * stride;
         if (u < units) {
-          int64_t local;
-          locate(p, u * VEC, cs[k], local);
+          locate(p, u * VEC, cs[k], locs[k]);
 #pragma unroll
-          for (int j = 0; j < TT; ++j) IO<Tin, VEC>::load(p.in[(cs[k] + 1 + j) % TT], u * VEC, v[k][j]);
+          for (int j = 0; j < TT; ++j)
+            raw[k][j] = ld_nc_v4(static_cast<const Tin*>(p.in[(cs[k] + 1 + j) % TT]) + u * VEC);
         }
       }
 #pragma unroll
@@ -198,17 +213,18 @@ __global__ void __launch_bounds__(256) ring_reduce_kernel(const __grid_constant_
         const int64_t u = u0 + k * stride;
         if (u >= units) break;
         float acc[VEC];
-#pragma unroll
-        for (int i = 0; i < VEC; ++i) acc[i] = v[k][0][i];
+        unpack16<Tin, VEC>(raw[k][0], acc);
 #pragma unroll
         for (int j = 1; j < TT; ++j) {
+          float v[VEC];
+          unpack16<Tin, VEC>(raw[k][j], v);
 #pragma unroll
           for (int i = 0; i < VEC; ++i) {
-            acc[i] = __fadd_rn(acc[i], v[k][j][i]);
+            acc[i] = __fadd_rn(acc[i], v[i]);
             if constexpr (HOP) acc[i] = hop_round(acc[i]);
           }
         }
-        finish_unit<Tout, VEC, AR>(p, u * VEC, cs[k], acc, t);
+        finish_unit<Tout, VEC, AR>(p, u * VEC, cs[k], locs[k], acc, t);
       }
     } else {
 #pragma unroll 1
@@ -230,7 +246,7 @@ __global__ void __launch_bounds__(256) ring_reduce_kernel(const __grid_constant_
             if constexpr (HOP) acc[i] = hop_round(acc[i]);
           }
         }
-        finish_unit<Tout, VEC, AR>(p, e, c, acc, t);
+        finish_unit<Tout, VEC, AR>(p, e, c, local, acc, t);
       }
     }
   }
@@ -354,10 +370,11 @@ int grid_for(int64_t units, int unr) {
   return static_cast<int>((threads + 255) / 256);
 }
 
-// Units per thread step: about 8 input vectors in flight per thread.
+// Units per thread step: 4-8 input vectors in flight per thread. Measured on one B200 against
+// 4 units for t = 2: 2 units were 3-8% faster at 64-256 MiB (fp32 and bf16), equal elsewhere.
 template <int TT>
 constexpr int unroll_for() {
-  return TT == 2 ? 4 : TT == 4 ? 2 : 1;
+  return TT == 2 || TT == 4 ? 2 : 1;
 }
 
 template <typename Tin, typename Tout, int VEC, bool AR, bool HOP = false>
@@ -403,7 +420,7 @@ tp_status ring_collective(const RingArgs& a, cudaStream_t stream) {
   if (hop && a.in_dtype != a.out_dtype) return fail(TP_EINVAL, "per-hop bf16 rounding needs bf16 in and out");
   if (!ring_dtype_ok(a.in_dtype) || !ring_dtype_ok(a.out_dtype)) return fail(TP_EINVAL, "bad dtype");
   if (a.op == RING_AG && a.in_dtype != a.out_dtype) return fail(TP_EINVAL, "AllGather copies bits: dtypes must match");
-  const int axis = a.op == RING_AR ? 0 : a.axis;
+  const int axis = a.axis;   // AllReduce: the axis of its ReduceScatter (each element's summation order)
   if (axis == 0 && a.rows % a.t) return fail(TP_EDIVIS, "t=%d does not divide rows=%lld", a.t, (long long)a.rows);
   if (axis == 1 && a.cols % a.t) return fail(TP_EDIVIS, "t=%d does not divide cols=%lld", a.t, (long long)a.cols);
   for (int i = 0; i < a.t; ++i)
@@ -438,14 +455,26 @@ tp_status ring_collective(const RingArgs& a, cudaStream_t stream) {
       in_place = static_cast<const char*>(a.in[i]) == static_cast<const char*>(a.out[i]) + i * p.chunk_elems * es;
     p.skip_self = in_place ? 1 : 0;
     const int64_t units = a.rows * a.cols / (vec ? epu : 1);
-    constexpr int G_UNR = 2;
-    const int blocks = grid_for(units, G_UNR);
+    // vectors per thread step: 4 for t = 2 (one store per vector and replica, few stores), 2
+    // otherwise (measured: 4 was 5% faster at t = 2 and 256 MiB, 1-2% slower at t = 8)
+    if (a.t <= 2) {
+      const int blocks = grid_for(units, 4);
+      if (es == 4) {
+        if (vec) ring_gather_kernel<4, 16, 4><<<blocks, 256, 0, stream>>>(p);
+        else ring_gather_kernel<4, 4, 4><<<blocks, 256, 0, stream>>>(p);
+      } else {
+        if (vec) ring_gather_kernel<2, 16, 4><<<blocks, 256, 0, stream>>>(p);
+        else ring_gather_kernel<2, 2, 4><<<blocks, 256, 0, stream>>>(p);
+      }
+      return check_launch("ring_gather_kernel");
+    }
+    const int blocks = grid_for(units, 2);
     if (es == 4) {
-      if (vec) ring_gather_kernel<4, 16, G_UNR><<<blocks, 256, 0, stream>>>(p);
-      else ring_gather_kernel<4, 4, G_UNR><<<blocks, 256, 0, stream>>>(p);
+      if (vec) ring_gather_kernel<4, 16, 2><<<blocks, 256, 0, stream>>>(p);
+      else ring_gather_kernel<4, 4, 2><<<blocks, 256, 0, stream>>>(p);
     } else {
-      if (vec) ring_gather_kernel<2, 16, G_UNR><<<blocks, 256, 0, stream>>>(p);
-      else ring_gather_kernel<2, 2, G_UNR><<<blocks, 256, 0, stream>>>(p);
+      if (vec) ring_gather_kernel<2, 16, 2><<<blocks, 256, 0, stream>>>(p);
+      else ring_gather_kernel<2, 2, 2><<<blocks, 256, 0, stream>>>(p);
     }
     return check_launch("ring_gather_kernel");
   }

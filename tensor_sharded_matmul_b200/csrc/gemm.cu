@@ -165,6 +165,14 @@ __device__ __forceinline__ bool produce_unit(const Ctl& c, Ring& r, const CUtens
                                              const CUtensorMap* b2, int m0, int n0, int num_kb, int* last_phase,
                                              bool* issued, int a_kslice = 0, int a_kslices = 1, int b_nslice = 0,
                                              int b_nslices = 1) {
+  // Slice views are chosen without divisions in the loop: B's four boxes once per unit, A's piece by
+  // counting k-blocks (the producer's per-stage latency paces the whole pipeline).
+  const CUtensorMap* bv[4];
+  int bn[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) bv[j] = slice_view(b, b_nslice, b_nslices, n0 + 64 * j, bn[j]);
+  const int a_kbs = a_kslice / BK;      // k-blocks per A piece (0: A not split along K)
+  int a_sl = 0, a_lk = 0;
   for (int kb = 0; kb < num_kb; ++kb) {
     if (!wait_or_abort(c, c.empty0 + 8 * r.stage, r.phase ^ 1u, WAIT_PRODUCER_EMPTY)) return false;
     const uint32_t fb = c.full0 + 8 * r.stage;
@@ -176,8 +184,13 @@ __device__ __forceinline__ bool produce_unit(const Ctl& c, Ring& r, const CUtens
       tma_load_2d(a_dst, a, m0, k0, fb);
       tma_load_2d(a_dst + B_BOX, a, m0 + 64, k0, fb);
     } else {                            // A [M][K]: one 64(K) x 128(M) box
-      int ak0;
-      const CUtensorMap* av = slice_view(a, a_kslice, a_kslices, k0, ak0);
+      const CUtensorMap* av = a;
+      int ak0 = k0;
+      if (a_kbs) {
+        if (a_lk == a_kbs && a_sl < a_kslices - 1) { ++a_sl; a_lk = 0; }
+        av = a + a_sl;
+        ak0 = a_lk++ * BK;
+      }
       tma_load_2d(a_dst, av, ak0, m0, fb);
     }
     // B (the weights) is re-read by every row-tile: the fused kernel keeps its lines in L2 longest
@@ -190,11 +203,7 @@ __device__ __forceinline__ bool produce_unit(const Ctl& c, Ring& r, const CUtens
       tma_load_2d_hint(b_dst + 3 * B_BOX, b2, n0 + 64, k0, fb, c.b_policy);
     } else {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        int bn;
-        const CUtensorMap* bv = slice_view(b, b_nslice, b_nslices, n0 + 64 * j, bn);
-        tma_load_2d_hint(b_dst + j * B_BOX, bv, bn, k0, fb, c.b_policy);
-      }
+      for (int j = 0; j < 4; ++j) tma_load_2d_hint(b_dst + j * B_BOX, bv[j], bn[j], k0, fb, c.b_policy);
     }
     issued[r.stage] = true;
     last_phase[r.stage] = static_cast<int>(r.phase);
@@ -549,6 +558,12 @@ __device__ __forceinline__ bool pair_produce_unit(const PairCtl& c, PairRing& r,
                                                   int a_kslice = 0, int a_kslices = 1, int b_nslice = 0,
                                                   int b_nslices = 1) {
   const uint32_t tx = 2 * (PAIR_A_STAGE + (wide ? PAIR_B_STAGE : PAIR_B_STAGE / 2));
+  // slice views without divisions in the loop (see produce_unit)
+  int bn0, bn1;
+  const CUtensorMap* bv0 = slice_view(tb, b_nslice, b_nslices, nb, bn0);
+  const CUtensorMap* bv1 = slice_view(tb, b_nslice, b_nslices, nb + 64, bn1);
+  const int a_kbs = a_kslice / BK;
+  int a_sl = 0, a_lk = 0;
   for (int kb = 0; kb < num_kb; kb += PAIR_KB) {
     if (!mbar_wait_bounded(c.empty0 + 8 * r.stage, r.phase ^ 1u, c.budget, c.abort_flag))
       return pair_fail(c, WAIT_PRODUCER_EMPTY);
@@ -563,20 +578,20 @@ __device__ __forceinline__ bool pair_produce_unit(const PairCtl& c, PairRing& r,
         tma_load_2d_pair(a_dst, ta, m0, k0, fb);
         tma_load_2d_pair(a_dst + B_BOX, ta, m0 + 64, k0, fb);
       } else {
-        int ak0;
-        const CUtensorMap* av = slice_view(ta, a_kslice, a_kslices, k0, ak0);
+        const CUtensorMap* av = ta;
+        int ak0 = k0;
+        if (a_kbs) {
+          if (a_lk == a_kbs && a_sl < a_kslices - 1) { ++a_sl; a_lk = 0; }
+          av = ta + a_sl;
+          ak0 = a_lk++ * BK;
+        }
         tma_load_2d_pair(a_dst, av, ak0, m0, fb);
       }
       if (c.b_km) {                     // B^T [N][K]: one 64(K) x 128(N) box of this CTA's columns
         tma_load_2d_pair_hint(b_dst, tb, k0, nb, fb, c.b_policy);
       } else {
-        int bn;
-        const CUtensorMap* bv = slice_view(tb, b_nslice, b_nslices, nb, bn);
-        tma_load_2d_pair_hint(b_dst, bv, bn, k0, fb, c.b_policy);
-        if (wide) {
-          bv = slice_view(tb, b_nslice, b_nslices, nb + 64, bn);
-          tma_load_2d_pair_hint(b_dst + B_BOX, bv, bn, k0, fb, c.b_policy);
-        }
+        tma_load_2d_pair_hint(b_dst, bv0, bn0, k0, fb, c.b_policy);
+        if (wide) tma_load_2d_pair_hint(b_dst + B_BOX, bv1, bn1, k0, fb, c.b_policy);
       }
     }
     r.advance();
@@ -1360,7 +1375,8 @@ tp_status ring_gemm(const RingGemmArgs& g, cudaStream_t s) {
   if (g.M == 0 || g.N == 0) return TP_OK;               // empty output: nothing to compute
   if (g.M > INT32_MAX / 2 || g.N > INT32_MAX / 2 || g.K > INT32_MAX / 2) return fail(TP_ESHAPE, "GEMM size too large");
   if (g.op != RING_RS && g.op != RING_AR) return fail(TP_EINVAL, "fused GEMM reduces by RS or AR only");
-  const int axis = g.op == RING_AR ? 0 : g.axis;
+  if (g.axis != 0 && g.axis != 1) return fail(TP_EINVAL, "axis must be 0 or 1");
+  const int axis = g.axis;              // AllReduce: the axis of its ReduceScatter (the summation order)
   if (!ring_gemm_fits(g.M, g.N, g.t, axis)) return fail(TP_EUNSUPPORTED, "chunks do not align with 128 x 256 tiles");
   if (g.K % 8 || g.N % 8 || g.lda % 8 || g.ldb % 8) return fail(TP_EALIGN, "K, N and row strides must be multiples of 8");
   if (g.lda < g.K || g.ldb < (g.b_km ? g.K : g.N)) return fail(TP_ESHAPE, "row stride shorter than the row");
@@ -1369,9 +1385,8 @@ tp_status ring_gemm(const RingGemmArgs& g, cudaStream_t s) {
     return fail(TP_EALIGN, "residual or bf16 copy not 16-byte aligned");
   RingGemmParams p;
   std::memset(&p, 0, sizeof(p));
-  const int axis0 = g.op == RING_AR ? 0 : g.axis;
-  const int64_t chunk0 = axis0 == 0 ? g.M / g.t : g.N / g.t;
-  const bool pair = axis0 == 0 ? chunk0 % (2 * BM) == 0 : g.M >= 2 * BM;
+  const int64_t chunk0 = axis == 0 ? g.M / g.t : g.N / g.t;
+  const bool pair = axis == 0 ? chunk0 % (2 * BM) == 0 : g.M >= 2 * BM;
   for (int i = 0; i < g.t; ++i) {
     if (!encode_bf16_2d(&p.ta[i], g.a[i], g.K, g.M, g.lda, BK, BM))
       return fail(TP_ECUDA, "cannot encode the TMA descriptor of A[%d]", i);

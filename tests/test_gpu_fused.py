@@ -64,6 +64,13 @@ CASES = [
     # axis 1 places no constraint on the row count: a partial last row-tile on the single-CTA kernel
     (2, 200, 512, 512, tp.TP_OUT_RS, 1),
     (4, 72, 256, 1024, tp.TP_OUT_RS, 1),
+    # AllReduce whose ReduceScatter runs along columns (each element summed in its column chunk's
+    # ring order): pairs, a 128-row M tail, the single-CTA kernel, the 70B W_O shape
+    (4, 512, 1024, 1024, tp.TP_OUT_AR, 1),
+    (2, 384, 512, 512, tp.TP_OUT_AR, 1),
+    (4, 200, 256, 1024, tp.TP_OUT_AR, 1),
+    (8, 2048, 1024, 4096, tp.TP_OUT_AR, 1),      # 8 x 16 tiles: more tiles than pairs, half-width round
+    (8, 2048, 8192, 8192, tp.TP_OUT_AR, 1),
 ]
 
 
@@ -78,8 +85,12 @@ def test_fused_equals_unfused_bitwise_and_oracle(t, N, k, n, mode, axis):
     plain = [torch.empty(shape, device="cuda") for _ in range(t)]
     if mode == tp.TP_OUT_RS:
         tp.tp_reduce_scatter(partials, plain, N, n, axis, tp.TP_F32, t)
-    else:
+    elif axis == 0:
         tp.tp_all_reduce(partials, plain, N, n, tp.TP_F32, t)
+    else:                   # AllReduce along columns = ReduceScatter(axis 1) then AllGather(axis 1)
+        pieces = [torch.empty((N, n // t), device="cuda") for _ in range(t)]
+        tp.tp_reduce_scatter(partials, pieces, N, n, 1, tp.TP_F32, t)
+        tp.tp_all_gather(pieces, plain, N, n, 1, tp.TP_F32, t)
     torch.cuda.synchronize()
     st, site = tp.tp_device_status(1)
     assert st == tp.TP_OK, f"device wait site {site}"
@@ -145,3 +156,18 @@ def test_unaligned_chunks_need_partials():
     Y = sum(OM.matmul(f64(x[r]), f64(w[r])) for r in range(t))
     for r in range(t):
         assert_close(f64(out[r]), Y[r * N // t:(r + 1) * N // t], GEMM_TOL, f"block {r}")
+
+
+@pytest.mark.parametrize("t,N,k,n", [(4, 256, 512, 520), (3, 96, 384, 264)])
+def test_unfused_all_reduce_along_columns(t, N, k, n):
+    # n/t is not a whole number of 256-column tiles: the partials path with the ring kernel's
+    # AllReduce along columns, bit-identical to ReduceScatter(axis 1) then AllGather(axis 1) and to
+    # the oracle's ring order fed the same partials
+    x, w = _operands(t, N, k, n, seed=31 + t)
+    out = [torch.empty((N, n), device="cuda") for _ in range(t)]
+    partials = [torch.empty((N, n), device="cuda") for _ in range(t)]
+    tp.tp_row_linear_reduce(x, N, k, n, t, w, tp.TP_OUT_AR, 1, out, partials)
+    torch.cuda.synchronize()
+    ref = OC.all_reduce([host_bits(p) for p in partials], axis=1)
+    for r in range(t):
+        assert same_bits(host_bits(out[r]), ref[r]), f"replica {r}"
