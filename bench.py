@@ -495,6 +495,35 @@ def _time_ms(fn, iters: int, warmup: int = 3) -> float:
     return a.elapsed_time(b) / iters
 
 
+def _time_graph_ms(fn, per_graph: int, replays: int = 5) -> float:
+    """Average device time of one fn() call, measured by replaying a CUDA graph that holds `per_graph`
+    back-to-back calls (CUDA events around the replays, after one warm-up replay). The host's per-call
+    cost (argument marshalling, launch) stays out of the measurement, which matters for payloads
+    whose kernels run for a few microseconds."""
+    import torch
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for _ in range(3):
+            fn()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for _ in range(per_graph):
+            fn()
+    graph.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(replays):
+        graph.replay()
+    b.record()
+    torch.cuda.synchronize()
+    del graph
+    return a.elapsed_time(b) / (replays * per_graph)
+
+
 def _iters_for(expected_ms: float, budget_ms: float = 60.0, lo: int = 5, hi: int = 200) -> int:
     return max(lo, min(hi, int(budget_ms / max(expected_ms, 1e-3))))
 
@@ -503,7 +532,7 @@ def collective_point(t: int, dt: str, mib: int, op: str) -> dict:
     """One point of the collective sweep: ReduceScatter / AllGather / AllReduce in ring order over t
     shard buffers resident in HBM. M = each shard's full buffer for RS/AR, the gathered tensor for AG.
     GB/s = algorithmic bytes / time: RS and AG (t+1)M, AR 2tM; ring_bus_gbs is the NCCL-style
-    (t-1)/t M (x2 for AR) over the same time."""
+    (t-1)/t M (x2 for AR) over the same time. Each point replays a CUDA graph of back-to-back calls."""
     import torch
     import tensor_sharded_matmul_b200 as tp
     es = 4 if dt == "f32" else 2
@@ -527,7 +556,8 @@ def collective_point(t: int, dt: str, mib: int, op: str) -> dict:
         else:
             fn = lambda: tp.tp_all_reduce(ins, outs, rows, cols, code, t)  # noqa: E731
             nbytes = 2 * t * mib * (1 << 20)
-    ms = _time_ms(fn, _iters_for(nbytes / 6.0e9, 200.0))
+    per_graph = max(2, min(100, int(20e-3 / max(nbytes / 6.0e12, 1e-6))))   # about 20 ms of work per replay
+    ms = _time_graph_ms(fn, per_graph)
     del ins, outs
     torch.cuda.empty_cache()
     gbs = nbytes / (ms * 1e-3) / 1e9
@@ -539,7 +569,7 @@ CASE_NAMES = {(1, 0): "local", (2, 0): "allgather", (2, 1): "allreduce", (3, 0):
               (3, 2): "rs_f", (4, 0): "gather_x", (4, 1): "gather_w"}
 
 
-def sharded_matmul_cases(which=None):
+def sharded_matmul_cases(which=None, iters=None):
     """The four sharded-matmul cases of C[B,F] = X[B,D] W[D,F] at B=D=8192, F=28672 over t=4 shards
     (`which`: the (case, strategy) pairs to time, default all). TFLOP/s counts the FLOPs executed
     (case 2 AllGather computes C on every shard). Yields (case, strategy, name, ms, tflops, ws_bytes)."""
@@ -563,7 +593,7 @@ def sharded_matmul_cases(which=None):
         wsb = torch.empty(max(nbytes, 256), dtype=torch.uint8, device="cuda")
         fn = lambda: tp.tp_sharded_matmul(case_id, strategy, xs, ws, B, D, F, t, c, tp.TP_F32, wsb, nbytes)  # noqa: E731
         flops = 2.0 * B * D * F * (t if (case_id, strategy) == (2, 0) else 1)
-        ms = _time_ms(fn, _iters_for(flops / 1.2e12, 60.0, lo=5, hi=50))
+        ms = _time_ms(fn, iters if iters else _iters_for(flops / 1.2e12, 60.0, lo=5, hi=50))
         yield case_id, strategy, name, ms, flops / (ms * 1e-3) / 1e12, nbytes
         del c, wsb, xs, ws
         torch.cuda.empty_cache()
@@ -668,7 +698,12 @@ def run_cases(args) -> int:
     import torch
     torch.cuda.set_device(0)
     peak = _peaks()[1]
-    for case_id, strategy, name, ms, rate, nbytes in sharded_matmul_cases():
+    which = None
+    if args.case:
+        c, st = (int(v) for v in args.case.split("."))
+        which = {(c, st)}
+    iters = args.steps if args.steps < 500 else None
+    for case_id, strategy, name, ms, rate, nbytes in sharded_matmul_cases(which, iters):
         _emit({"config": "sharded_matmul", "case": case_id, "strategy": name, "ms": ms, "tflops_executed": rate,
                "frac_bf16_peak": rate / peak, "workspace_bytes": nbytes})
     return 0
@@ -691,6 +726,8 @@ ROW_REDUCE_SHAPES = {
     "70b_wo_ar": (8, 2048, 8192, 8192, "AR"),        # Llama-3-70B attention output projection + AR
     "70b_down_ar": (8, 2048, 28672, 8192, "AR"),     # Llama-3-70B down projection + AR
 }
+# chunk axis of each shape's ReduceScatter: the 70B layer's AllReduces scatter along h (columns)
+ROW_REDUCE_AXIS = {"8b_rs_ag": 0, "8b_rs": 0, "70b_wo_ar": 1, "70b_down_ar": 1}
 
 
 def run_rowreduce(args) -> int:
@@ -711,10 +748,12 @@ def run_rowreduce(args) -> int:
         w = d.normal((t, k // t, n), 0.02)
         rows = N // t if mode == "RS" else N
         out = [torch.empty((rows, n), device="cuda") for _ in range(t)]
-        fn = lambda: tp.tp_row_linear_reduce(x, N, k, n, t, w, modes[mode], 0, out)  # noqa: E731
+        axis = ROW_REDUCE_AXIS[name]
+        fn = lambda: tp.tp_row_linear_reduce(x, N, k, n, t, w, modes[mode], axis, out)  # noqa: E731
         ms = _time_ms(fn, args.steps if args.steps < 500 else 50)
         rate = 2.0 * N * k * n / (ms * 1e-3) / 1e12
-        _emit({"config": "rowreduce", "shape": name, "t": t, "tokens": N, "k": k, "n": n, "mode": mode, "ms": ms,
+        _emit({"config": "rowreduce", "shape": name, "t": t, "tokens": N, "k": k, "n": n, "mode": mode, "axis": axis,
+               "ms": ms,
                "tflops": rate, "frac_bf16_peak": rate / burst,
                "bytes_written": t * rows * n * 4})
         del x, w, out
@@ -803,6 +842,7 @@ def main(argv=None) -> int:
                     help="time the headline step only (profiling runs; multi-GPU runs always do)")
     ap.add_argument("--config", choices=["mlp8b", "sweep", "cases", "layer70b", "next", "rowreduce"], default="mlp8b",
                     help="mlp8b: the headline step (one JSON line); the others print one line per measurement")
+    ap.add_argument("--case", default=None, help="--config cases: one strategy only, as CASE.STRATEGY (e.g. 4.1)")
     ap.add_argument("--shape", choices=sorted(ROW_REDUCE_SHAPES), default=None,
                     help="--config rowreduce: one shape only (default: all)")
     args = ap.parse_args(argv)
