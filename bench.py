@@ -528,11 +528,17 @@ def _iters_for(expected_ms: float, budget_ms: float = 60.0, lo: int = 5, hi: int
     return max(lo, min(hi, int(budget_ms / max(expected_ms, 1e-3))))
 
 
+L2_BYTES = 126 * 2**20   # B200 L2
+
+
 def collective_point(t: int, dt: str, mib: int, op: str) -> dict:
     """One point of the collective sweep: ReduceScatter / AllGather / AllReduce in ring order over t
     shard buffers resident in HBM. M = each shard's full buffer for RS/AR, the gathered tensor for AG.
     GB/s = algorithmic bytes / time: RS and AG (t+1)M, AR 2tM; ring_bus_gbs is the NCCL-style
-    (t-1)/t M (x2 for AR) over the same time. Each point replays a CUDA graph of back-to-back calls."""
+    (t-1)/t M (x2 for AR) over the same time. Each point replays a CUDA graph of back-to-back calls
+    (the host's per-call cost stays out), and the calls cycle through enough independent buffer sets
+    that about twice the L2's size streams between two uses of a set: small payloads are timed from
+    HBM, not from L2."""
     import torch
     import tensor_sharded_matmul_b200 as tp
     es = 4 if dt == "f32" else 2
@@ -541,28 +547,39 @@ def collective_point(t: int, dt: str, mib: int, op: str) -> dict:
     elems = mib * (1 << 20) // es
     cols = 4096 if elems >= 4096 * 64 else 256
     rows = elems // cols
-    if op == "AG":
-        ins = [torch.empty((rows // t, cols), dtype=tdt, device="cuda").normal_() for _ in range(t)]
-        outs = [torch.empty((rows, cols), dtype=tdt, device="cuda") for _ in range(t)]
-        fn = lambda: tp.tp_all_gather(ins, outs, rows, cols, 0, code, t)  # noqa: E731
-        nbytes = (t + 1) * mib * (1 << 20)
-    else:
-        ins = [torch.empty((rows, cols), dtype=tdt, device="cuda").normal_() for _ in range(t)]
-        shape = (rows // t, cols) if op == "RS" else (rows, cols)
-        outs = [torch.empty(shape, dtype=tdt, device="cuda") for _ in range(t)]
-        if op == "RS":
-            fn = lambda: tp.tp_reduce_scatter(ins, outs, rows, cols, 0, code, t)  # noqa: E731
-            nbytes = (t + 1) * mib * (1 << 20)
+    M = mib * (1 << 20)
+    footprint = {"RS": (t + 1) * M, "AG": (t + 1) * M, "AR": 2 * t * M}[op]
+    nsets = max(1, min(128, -(-2 * L2_BYTES // footprint)))
+    sets = []
+    for _ in range(nsets):
+        if op == "AG":
+            ins = [torch.empty((rows // t, cols), dtype=tdt, device="cuda").normal_() for _ in range(t)]
+            outs = [torch.empty((rows, cols), dtype=tdt, device="cuda") for _ in range(t)]
         else:
-            fn = lambda: tp.tp_all_reduce(ins, outs, rows, cols, code, t)  # noqa: E731
-            nbytes = 2 * t * mib * (1 << 20)
-    per_graph = max(2, min(100, int(20e-3 / max(nbytes / 6.0e12, 1e-6))))   # about 20 ms of work per replay
+            ins = [torch.empty((rows, cols), dtype=tdt, device="cuda").normal_() for _ in range(t)]
+            shape = (rows // t, cols) if op == "RS" else (rows, cols)
+            outs = [torch.empty(shape, dtype=tdt, device="cuda") for _ in range(t)]
+        sets.append((ins, outs))
+    nbytes = footprint
+    calls = {"RS": lambda i, o: tp.tp_reduce_scatter(i, o, rows, cols, 0, code, t),
+             "AG": lambda i, o: tp.tp_all_gather(i, o, rows, cols, 0, code, t),
+             "AR": lambda i, o: tp.tp_all_reduce(i, o, rows, cols, code, t)}[op]
+    state = {"k": 0}
+
+    def fn():
+        i, o = sets[state["k"] % nsets]
+        state["k"] += 1
+        calls(i, o)
+
+    per_graph = max(2, min(128, int(20e-3 / max(nbytes / 6.0e12, 1e-6))))   # about 20 ms of work per replay
+    per_graph = nsets * max(1, -(-per_graph // nsets))                       # every set equally often
     ms = _time_graph_ms(fn, per_graph)
-    del ins, outs
+    del sets
     torch.cuda.empty_cache()
     gbs = nbytes / (ms * 1e-3) / 1e9
-    bus = (t - 1) / t * mib * (1 << 20) * (2 if op == "AR" else 1) / (ms * 1e-3) / 1e9
-    return {"ms": ms, "gbs": gbs, "frac_hbm": gbs / _peaks()[0], "ring_bus_gbs": bus, "bytes": nbytes}
+    bus = (t - 1) / t * M * (2 if op == "AR" else 1) / (ms * 1e-3) / 1e9
+    return {"ms": ms, "gbs": gbs, "frac_hbm": gbs / _peaks()[0], "ring_bus_gbs": bus, "bytes": nbytes,
+            "buffer_sets": nsets}
 
 
 CASE_NAMES = {(1, 0): "local", (2, 0): "allgather", (2, 1): "allreduce", (3, 0): "allreduce", (3, 1): "rs_b",
@@ -748,7 +765,7 @@ def run_rowreduce(args) -> int:
         w = d.normal((t, k // t, n), 0.02)
         rows = N // t if mode == "RS" else N
         out = [torch.empty((rows, n), device="cuda") for _ in range(t)]
-        axis = ROW_REDUCE_AXIS[name]
+        axis = ROW_REDUCE_AXIS[name] if args.axis is None else args.axis
         fn = lambda: tp.tp_row_linear_reduce(x, N, k, n, t, w, modes[mode], axis, out)  # noqa: E731
         ms = _time_ms(fn, args.steps if args.steps < 500 else 50)
         rate = 2.0 * N * k * n / (ms * 1e-3) / 1e12
@@ -842,6 +859,8 @@ def main(argv=None) -> int:
                     help="time the headline step only (profiling runs; multi-GPU runs always do)")
     ap.add_argument("--config", choices=["mlp8b", "sweep", "cases", "layer70b", "next", "rowreduce"], default="mlp8b",
                     help="mlp8b: the headline step (one JSON line); the others print one line per measurement")
+    ap.add_argument("--axis", type=int, choices=[0, 1], default=None,
+                    help="--config rowreduce: chunk axis of the ReduceScatter (default: the shape's own)")
     ap.add_argument("--case", default=None, help="--config cases: one strategy only, as CASE.STRATEGY (e.g. 4.1)")
     ap.add_argument("--shape", choices=sorted(ROW_REDUCE_SHAPES), default=None,
                     help="--config rowreduce: one shape only (default: all)")

@@ -300,6 +300,67 @@ def test_cases_full_size_sampled(case_operands_full, case_id, strategy):
 
 
 # ---------------------------------------------------------------------------------- 70B-shaped layer
+def _layer_device(L, N, h, n_h, n_kv, d_h, F, t, with_partials):
+    d = {k: cuda(v) for k, v in L.items()}
+    kv = n_kv // t if t <= n_kv else 1
+    qkv_w = (n_h // t + 2 * kv) * d_h
+    w_qkv = torch.empty((t, h, qkv_w), dtype=torch.bfloat16, device="cuda")
+    w_o = torch.empty((t, n_h * d_h // t, h), dtype=torch.bfloat16, device="cuda")
+    w_gu = torch.empty((t, h, 2 * F // t), dtype=torch.bfloat16, device="cuda")
+    w_down = torch.empty((t, F // t, h), dtype=torch.bfloat16, device="cuda")
+    tp.tp_shard_qkv(d["Wq"], n_h * d_h, d["Wk"], n_kv * d_h, d["Wv"], n_kv * d_h, h, n_h, n_kv, d_h, t, w_qkv)
+    tp.tp_shard_rows(d["Wo"], h, n_h * d_h, h, t, w_o)
+    tp.tp_shard_gate_up(d["Wg"], F, d["Wu"], F, h, F, t, w_gu)
+    tp.tp_shard_rows(d["Wd"], h, F, h, t, w_down)
+    o_shards = [d["O"][:, r * n_h * d_h // t:(r + 1) * n_h * d_h // t].contiguous() for r in range(t)]
+    out = dict(qkv=torch.empty((t, N, qkv_w), dtype=torch.bfloat16, device="cuda"),
+               h1=[torch.empty((N, h), device="cuda") for _ in range(t)],
+               h1_bf16=torch.empty((N, h), dtype=torch.bfloat16, device="cuda"),
+               y=[torch.empty((N, h), device="cuda") for _ in range(t)])
+    z_ws = torch.empty((t, N, F // t), dtype=torch.bfloat16, device="cuda")
+    partials = [torch.empty((N, h), device="cuda") for _ in range(t)] if with_partials else None
+    tp.tp_layer_fwd(d["X"], o_shards, N, h, n_h, n_kv, d_h, F, t, w_qkv, w_o, w_gu, w_down, out["qkv"], out["h1"],
+                    out["h1_bf16"], z_ws, partials, out["y"])
+    torch.cuda.synchronize()
+    _status_ok()
+    return out
+
+
+def _layer_oracle(L, n_h, n_kv, d_h, t, rows=None):
+    f32 = lambda x: x.float().numpy()  # noqa: E731  (exact widening of bf16)
+    sh_qkv = OL.shard_qkv(f32(L["Wq"]), f32(L["Wk"]), f32(L["Wv"]), n_h, n_kv, d_h, t)
+    sh_o = OL.shard_rows(f32(L["Wo"]), t)
+    sh_gu = OL.shard_gate_up(f32(L["Wg"]), f32(L["Wu"]), t)
+    sh_d = OL.shard_rows(f32(L["Wd"]), t)
+    O = f32(L["O"])
+    O_sh = [O[:, r * n_h * d_h // t:(r + 1) * n_h * d_h // t] for r in range(t)]
+    return OLAYER.layer_forward(f32(L["X"]), O_sh, list(sh_qkv), list(sh_o), list(sh_gu), list(sh_d), rows=rows)
+
+
+# The layer's two AllReduces run fused with their row GEMMs, scattering along h when h/t is whole
+# 256-column tiles (first shape), else along tokens when N/t is whole 128-row tiles (second), else
+# unfused through the partials (third). Every path is compared in full with the fp64 oracle.
+@pytest.mark.parametrize("N,h,n_h,n_kv,d_h,F,t,with_partials", [
+    (256, 1024, 16, 4, 64, 2048, 4, False),
+    (512, 512, 8, 4, 64, 1024, 4, False),
+    (96, 512, 8, 2, 64, 1024, 4, True),
+])
+def test_layer_small_every_reduction_path(N, h, n_h, n_kv, d_h, F, t, with_partials):
+    L = S.llama70b_layer(seed=3, N=N, h=h, n_h=n_h, n_kv=n_kv, d_h=d_h, F=F)
+    got = _layer_device(L, N, h, n_h, n_kv, d_h, F, t, with_partials)
+    ref = _layer_oracle(L, n_h, n_kv, d_h, t)
+    for r in range(t):
+        assert_close(f64(got["qkv"][r]), ref["qkv"][r], GEMM_TOL, f"qkv {r}")
+    for s in range(t):
+        assert_close(f64(got["h1"][s]), ref["h1"], GEMM_TOL, f"h1 replica {s}")
+        assert_close(f64(got["y"][s]), ref["y"], GEMM_TOL, f"y replica {s}")
+        assert same_bits(host_bits(got["h1"][s]), host_bits(got["h1"][0]))
+        assert same_bits(host_bits(got["y"][s]), host_bits(got["y"][0]))
+    # the MLP's input is h1 rounded once to bf16
+    assert np.array_equal(host_bits(got["h1_bf16"]), f32_to_bf16_bits(host_bits(got["h1"][0])))
+    assert_close(f64(got["y"][0]) - f64(got["h1"][0]), ref["mlp"], GEMM_TOL, "mlp part")
+
+
 def test_llama70b_layer_sampled_rows():
     N, h, n_h, n_kv, d_h, F, t = 2048, 8192, 64, 8, 128, 28672, 8
     L = S.llama70b_layer(seed=0)
