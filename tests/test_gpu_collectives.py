@@ -216,7 +216,8 @@ def test_all_to_all_moves_the_sharded_dim():
 
 # ---------------------------------------------------------------------------------- per-hop bf16 mode
 @pytest.mark.parametrize("t,rows,cols,axis", [(2, 64, 256, 0), (3, 96, 72, 0), (4, 64, 256, 1), (8, 512, 4096, 0),
-                                              (5, 40, 80, 1), (3, 9, 7, 0), (4, 1028, 4104, 0)])
+                                              (5, 40, 80, 1), (3, 9, 7, 0), (4, 1028, 4104, 0), (16, 256, 512, 0),
+                                              (16, 64, 1024, 1), (1, 8, 16, 0)])
 def test_per_hop_bf16_reduce_scatter_and_all_reduce_bit_exact(t, rows, cols, axis):
     ins = _payload(t, rows, cols, "bf16", seed=900 + t * rows + cols)
     d_in = [cuda(x) for x in ins]

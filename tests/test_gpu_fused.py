@@ -71,6 +71,8 @@ CASES = [
     (4, 200, 256, 1024, tp.TP_OUT_AR, 1),
     (8, 2048, 1024, 4096, tp.TP_OUT_AR, 1),      # 8 x 16 tiles: more tiles than pairs, half-width round
     (8, 2048, 8192, 8192, tp.TP_OUT_AR, 1),
+    (1, 256, 256, 512, tp.TP_OUT_AR, 1),         # a single chunk
+    (16, 512, 2048, 4096, tp.TP_OUT_AR, 1),      # the maximum shard count, 256-column chunks
 ]
 
 
