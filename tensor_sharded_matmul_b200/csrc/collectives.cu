@@ -12,8 +12,10 @@
 //   AllGather: reads M, writes t*M.
 //   AllToAll (a bit copy, "Scaling Book 入门第 5 章", §5.3): reads t*M, writes t*M.
 // No atomics, no reassociation, and the result does not depend on grid size.
-// Memory traffic is coalesced 16-byte vectors; grids are a multiple of the SM count with
-// grid-stride loops. bf16 inputs are widened (exact), summed in binary32 and rounded once to bf16
+// A thread's unit is one 16-byte vector of the input type, so every warp-wide load is 32 consecutive
+// vectors; a thread takes a few units a grid stride apart and issues all their loads before any add,
+// and grids give every thread the same number of steps. bf16 inputs are widened (exact), summed in
+// binary32 and rounded once to bf16
 // (nearest-even) at the end; the optional per-hop mode (TP_BF16_RING) instead rounds the running
 // partial to bf16 after every add, as a ring whose links carry bf16 does.
 #include <cuda_bf16.h>

@@ -7,7 +7,10 @@
 //    column-parallel GEMM Z_r = act(X W_r), the row-parallel GEMM U_r = Z_r W_r when the partials
 //    themselves are wanted ("张量并行与序列并行", §矩阵乘法的两种切法 and §MLP：先列后行，只通信一次),
 //    and the local products of the sharded-matmul cases ("Scaling Book 入门第 6 章", §6.2). All t
-//    shards of one layer run in ONE launch over the tile space (shard, m-tile, n-tile).
+//    shards of one layer run in ONE launch over the tile space (shard, m-tile, n-tile). An operand
+//    may be given as the t pieces of an AllGather, each box read from the piece that holds it: A's
+//    row pieces (TP+SP input, case 4 gather X), A's K pieces (case 2 AllGather) or B's column pieces
+//    (case 4 gather W). The gather then never reaches memory ("Scaling Book 入门第 6 章", §6.6).
 //
 //  gemm_ring_kernel / gemm_ring_pair_kernel: the row-parallel GEMM fused with its collective, the
 //    one-GPU form of the pages' collective matmul ("Scaling Book 入门第 6 章", §6.6;
@@ -16,7 +19,8 @@
 //    c) into alternating TMEM accumulators. The epilogue adds them into an fp32 running sum in
 //    registers, one binary32 add per shard, which is exactly the ReduceScatter's summation order. It
 //    then writes the tile once: to shard c's output (ReduceScatter) or to all t outputs (AllReduce =
-//    ReduceScatter followed by AllGather), optionally adding a residual and writing a bf16 copy. The
+//    ReduceScatter followed by AllGather, its chunks rows or columns), optionally adding a residual
+//    and writing a bf16 copy. The
 //    fp32 partials never reach HBM. Each U_s tile comes from the same MMA instruction sequence as the
 //    plain GEMM's, so the results are bit-identical to the unfused GEMM followed by the ring kernel.
 //
