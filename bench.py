@@ -653,11 +653,53 @@ def layer70b():
     return ms, flops / 1e9
 
 
+def mlp_backward_ms(X, w_in, w_down, z, iters: int) -> float:
+    """CUDA-event ms per call of the Llama-3-8B TP-MLP backward (t=8, SwiGLU) from the forward's own
+    bf16 intermediates (H recomputed here, Z into z): dZ, dW_down, the SwiGLU backward, dW_in, and dX
+    with its ring AllReduce fused into the GEMM."""
+    import torch
+    import synthetic as S
+    import tensor_sharded_matmul_b200 as tp
+    t, N, h, f = T, N_TOK, H, F // T
+    bf16 = torch.bfloat16
+    dY = S.Draw(1, "cuda").normal((N, h), 1.0)
+    h_pre = torch.empty((t, N, 2 * f), dtype=bf16, device="cuda")
+    tp.tp_column_linear(X, N, h, 2 * F, t, tp.TP_ACT_NONE, w_in, h_pre)
+    tp.tp_column_linear(X, N, h, F, t, tp.TP_ACT_SWIGLU, w_in, z)
+    dz = torch.empty((t, N, f), dtype=bf16, device="cuda")
+    dh = torch.empty((t, N, 2 * f), dtype=bf16, device="cuda")
+    g_in = torch.empty((t, h, 2 * f), device="cuda")
+    g_down = torch.empty((t, f, h), device="cuda")
+    gx = [torch.empty((N, h), device="cuda") for _ in range(t)]
+    ms = _time_ms(lambda: tp.tp_mlp_bwd(X, dY, N, h, F, t, tp.TP_ACT_SWIGLU, w_in, w_down, h_pre, z, dz, dh, g_in,
+                                        g_down, gx), iters)
+    st, site = tp.tp_device_status(1)
+    if st != tp.TP_OK:
+        raise RuntimeError(f"device wait ran out at site {site}")
+    del h_pre, dz, dh, g_in, g_down, gx, dY
+    torch.cuda.empty_cache()
+    return ms
+
+
+def all_to_all_ms(iters: int) -> tuple[float, int]:
+    """CUDA-event ms per AllToAll over 8 fp32 [4096, 4096] shard buffers (split rows, concatenate
+    columns), and the bytes a bit copy must move (read t*M, write t*M)."""
+    import torch
+    import tensor_sharded_matmul_b200 as tp
+    t, N, h = T, N_TOK, H
+    ins = [torch.empty((N, h), device="cuda").normal_() for _ in range(t)]
+    outs = [torch.empty((N // t, t * h), device="cuda") for _ in range(t)]
+    ms = _time_ms(lambda: tp.tp_all_to_all(ins, outs, N, h, 0, 1, tp.TP_F32, t), iters)
+    del ins, outs
+    torch.cuda.empty_cache()
+    return ms, 2 * t * M_PARTIAL
+
+
 def workloads(X, w_in, w_down, z) -> dict:
     """The other workloads, each timed with CUDA events on the current stream after warm-up, under one
-    nvidia-smi clock record: the 70B layer, every sharded-matmul strategy, the TP+SP MLP forward on the
-    8B shape (reusing the headline step's weights) and the ring collectives at t in {2, 8}, fp32/bf16,
-    64 MiB and 1 GiB. Fractions are of the measured burst peaks (each kernel is timed in a short loop)."""
+    nvidia-smi clock record: the TP+SP MLP forward, the MLP backward and AllToAll on the 8B shape
+    (reusing the headline step's weights), the 70B layer, every sharded-matmul strategy and the ring
+    collectives at t in {2, 8}, fp32/bf16, 64 MiB and 1 GiB. Fractions are of the measured burst peaks (each kernel is timed in a short loop)."""
     import torch
     import tensor_sharded_matmul_b200 as tp
     hbm, burst, _, src = _peaks()
@@ -675,6 +717,12 @@ def workloads(X, w_in, w_down, z) -> dict:
     rate = FLOPS_STEP / (ms * 1e-3) / 1e12
     out["tp_sp_mlp_fwd_llama8b"] = {"ms": ms, "tflops": rate, "frac_bf16_peak": rate / burst}
     del x_shards, out_sp
+    ms = mlp_backward_ms(X, w_in, w_down, z, 20)
+    rate = 2 * FLOPS_STEP / (ms * 1e-3) / 1e12
+    out["mlp_bwd_llama8b"] = {"ms": ms, "tflops": rate, "frac_bf16_peak": rate / burst}
+    ms, nbytes = all_to_all_ms(50)
+    out["all_to_all_t8_f32_64MiB"] = {"ms": ms, "gbs": nbytes / (ms * 1e-3) / 1e9,
+                                      "frac_hbm": nbytes / (ms * 1e-3) / 1e9 / hbm}
     ms, gflop = layer70b()
     rate = gflop / ms
     out["llama70b_tp8_layer"] = {"ms": ms, "tflops": rate, "frac_bf16_peak": rate / burst, "gflop": gflop}
@@ -820,31 +868,11 @@ def run_next(args) -> int:
     del out_sp, x_shards
 
     # f3: backward, from the forward's own intermediates
-    d = S.Draw(1, "cuda")
-    dY = d.normal((N, h), 1.0)
-    h_pre = torch.empty((t, N, 2 * f), dtype=bf16, device="cuda")
-    tp.tp_column_linear(X, N, h, 2 * F, t, tp.TP_ACT_NONE, w_in, h_pre)
-    tp.tp_column_linear(X, N, h, F, t, tp.TP_ACT_SWIGLU, w_in, z)
-    dz = torch.empty((t, N, f), dtype=bf16, device="cuda")
-    dh = torch.empty((t, N, 2 * f), dtype=bf16, device="cuda")
-    g_in = torch.empty((t, h, 2 * f), device="cuda")
-    g_down = torch.empty((t, f, h), device="cuda")
-    gx = [torch.empty((N, h), device="cuda") for _ in range(t)]
-    ms = _time_ms(lambda: tp.tp_mlp_bwd(X, dY, N, h, F, t, tp.TP_ACT_SWIGLU, w_in, w_down, h_pre, z, dz, dh, g_in,
-                                        g_down, gx), 20)
+    ms = mlp_backward_ms(X, w_in, w_down, z, 20)
     tensor_line("f3 MLP backward (dZ, dW_down, SwiGLU backward, dW_in, dX + ring AllReduce)", ms, 2 * FLOPS_STEP)
-    st, site = tp.tp_device_status(1)
-    if st != tp.TP_OK:
-        print(f"device wait ran out at site {site}", file=sys.stderr)
-        return 3
-    del h_pre, dz, dh, g_in, g_down, gx, dY
-    torch.cuda.empty_cache()
 
     # f4: AllToAll, split rows / concatenate columns
-    ins = [torch.empty((N, h), device="cuda").normal_() for _ in range(t)]
-    outs = [torch.empty((N // t, t * h), device="cuda") for _ in range(t)]
-    ms = _time_ms(lambda: tp.tp_all_to_all(ins, outs, N, h, 0, 1, tp.TP_F32, t), 50)
-    nbytes = 2 * t * M_PARTIAL
+    ms, nbytes = all_to_all_ms(50)
     gbs = nbytes / (ms * 1e-3) / 1e9
     _emit({"config": "next", "row": "f4 AllToAll, 8 x fp32 [4096,4096], split rows / concat columns", "ms": ms,
            "gbs": gbs, "frac_hbm": gbs / hbm, "bytes": nbytes})

@@ -129,10 +129,11 @@ def mlp_backward(X, W_in_shards, W_out_shards, dY, act: str):
     ("张量并行与序列并行", §矩阵乘法的两种切法: column-parallel backward needs an AllReduce of dX, and
     row-parallel backward is local; pufanyi.com "ml-revisit-infra", §Tensor Parallel: dW_i = X^T dY_i,
     dX = sum_i dY_i W_i^T, and for the row split dW_i = X_i^T dY, dX_i = dY W_i^T).
-    Returns dX (the sum over shards), its per-shard partials, and dW_in / dW_out per shard."""
+    Returns dX (the sum over shards), its per-shard partials, dW_in / dW_out and the
+    pre-activation gradient dH per shard."""
     X = np.asarray(X, dtype=np.float64)
     dY = np.asarray(dY, dtype=np.float64)
-    out = {"dX_partials": [], "dW_in": [], "dW_out": []}
+    out = {"dX_partials": [], "dW_in": [], "dW_out": [], "dH": []}
     for W_in, W_out in zip(W_in_shards, W_out_shards):
         W_in = np.asarray(W_in, dtype=np.float64)
         W_out = np.asarray(W_out, dtype=np.float64)
@@ -147,6 +148,7 @@ def mlp_backward(X, W_in_shards, W_out_shards, dY, act: str):
             dH = np.concatenate([dZ * u * s * (1.0 + g * (1.0 - s)), dZ * g * s], axis=1)
         else:
             dH = dZ * act_derivative(H, act)
+        out["dH"].append(dH)
         out["dW_in"].append(X.T @ dH)           # column layer: weight gradient, local
         out["dX_partials"].append(dH @ W_in.T)  # column layer: input gradient, a partial sum
     out["dX"] = sum(out["dX_partials"])

@@ -52,6 +52,8 @@ def _forward_intermediates(dX, dw_in, N, h, F, t, act):
     (1024, 512, 2048, 4, "swiglu"),    # dX through the fused ring GEMM (CTA pairs)
     (1024, 1024, 4096, 8, "swiglu"),
     (256, 128, 512, 2, "none"),
+    (384, 256, 1088, 8, "swiglu"),     # F/t = 136: a partial 32-column chunk; a partial pair tile
+    (200, 128, 544, 4, "gelu"),        # one-CTA kernel, ragged rows and columns
 ])
 def test_mlp_backward_against_oracle(N, h, F, t, act):
     d = S.Draw(N + h + t)
@@ -74,6 +76,8 @@ def test_mlp_backward_against_oracle(N, h, F, t, act):
     assert st == tp.TP_OK, f"device wait site {site}"
     ref = OM.mlp_backward(f64(X), [f64(w) for w in w_in], [f64(w) for w in w_down], f64(dY), act)
     for r in range(t):
+        # dH_r from the activation's backward kernel (bf16); the GPU's H is its own bf16 forward
+        assert_close(f64(dh[r]), ref["dH"][r], GEMM_TOL, f"dH[{r}]")
         assert_close(f64(g_down[r]), ref["dW_out"][r], GEMM_TOL, f"dW_down[{r}]")
         assert_close(f64(g_in[r]), ref["dW_in"][r], GEMM_TOL, f"dW_in[{r}]")
         assert_close(f64(gx[r]), ref["dX"], GEMM_TOL, f"dX replica {r}")
