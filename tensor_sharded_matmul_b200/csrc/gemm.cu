@@ -61,7 +61,8 @@ constexpr uint32_t A_STAGE = BM * BK * 2;        // 16 KiB
 constexpr uint32_t B_STAGE = BN * BK * 2;        // 32 KiB
 constexpr uint32_t B_BOX = 64 * BK * 2;          // one 64(N) x 64(K) box, 8 KiB
 constexpr uint32_t TMEM_COLS = 512;              // two 128 x 256 fp32 accumulators
-constexpr int RASTER_BAND = 16;                  // row-tiles per raster band
+constexpr int RASTER_BAND_MAX = 16;              // row-tiles per raster band, at most
+constexpr int64_t RASTER_A_BYTES = 32ll << 20;   // A rows one band keeps in L2 while its B panels stream
 
 constexpr int GEMM_THREADS = 192;                // producer, MMA, 4 epilogue warps
 constexpr int RING_THREADS = 320;                // producer, MMA, 8 epilogue warps
@@ -264,13 +265,13 @@ __device__ __forceinline__ void teardown(const Ctl& c, int warp, int lane, const
   if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
 }
 
-// Tile index -> (row-tile, n-tile). Row-tiles form one sequence; it is cut into bands of
-// RASTER_BAND row-tiles and each band is swept across all n-tiles, row-tile fastest.
-__device__ __forceinline__ void raster(int tile, int row_tiles, int tiles_n, int& rt, int& nt) {
-  const int band_tiles = RASTER_BAND * tiles_n;
+// Tile index -> (row-tile, n-tile). Row-tiles form one sequence; it is cut into bands of `band_rows`
+// row-tiles and each band is swept across all n-tiles, row-tile fastest.
+__device__ __forceinline__ void raster(int tile, int row_tiles, int tiles_n, int band_rows, int& rt, int& nt) {
+  const int band_tiles = band_rows * tiles_n;
   const int band = tile / band_tiles;
-  const int first = band * RASTER_BAND;
-  const int in_band = min(RASTER_BAND, row_tiles - first);
+  const int first = band * band_rows;
+  const int in_band = min(band_rows, row_tiles - first);
   const int local = tile - band * band_tiles;
   rt = first + local % in_band;
   nt = local / in_band;
@@ -325,6 +326,7 @@ struct GemmParams {
   // column-split weight): column n of B is column n % b_nslice of tb[n / b_nslice]. 0 = not sliced.
   int b_nslice, b_nslices;
   int n_amaps, n_bmaps;             // tensor maps in ta[] / tb[] (prefetched at start)
+  int band;                         // row-tiles per raster band
   bool a_mn, b_km;                  // A stored [K][M] / B stored [N][K] (transposed operands)
   uint32_t* status;
   unsigned long long budget;
@@ -413,7 +415,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tcgen05_kernel(const __g
       Ring r;
       for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
         int rt, nt;
-        raster(tile, p.row_tiles, p.tiles_n, rt, nt);
+        raster(tile, p.row_tiles, p.tiles_n, p.band, rt, nt);
         const int g = rt / p.tiles_m;
         const int m0 = (rt - g * p.tiles_m) * BM;
         int am0;
@@ -444,7 +446,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tcgen05_kernel(const __g
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
       int rt, nt;
-      raster(tile, p.row_tiles, p.tiles_n, rt, nt);
+      raster(tile, p.row_tiles, p.tiles_n, p.band, rt, nt);
       const int g = rt / p.tiles_m;
       const int m0 = (rt - g * p.tiles_m) * BM;
       const int n0 = nt * TILE_N;
@@ -713,7 +715,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
       PairRing r;
       for (int tile = pair; tile < num_tiles; tile += pairs) {
         int rt, nt;
-        raster(tile, row_tiles, p.tiles_n, rt, nt);
+        raster(tile, row_tiles, p.tiles_n, p.band, rt, nt);
         const int g = rt / tiles_m;
         const int m0 = (rt - g * tiles_m) * TILE_M + static_cast<int>(c.rank) * BM;
         const int n0 = nt * TILE_N;
@@ -744,7 +746,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     uint32_t acc_phase = 0;
     for (int tile = pair; tile < num_tiles; tile += pairs) {
       int rt, nt;
-      raster(tile, row_tiles, p.tiles_n, rt, nt);
+      raster(tile, row_tiles, p.tiles_n, p.band, rt, nt);
       const int g = rt / tiles_m;
       const int m0 = (rt - g * tiles_m) * TILE_M + static_cast<int>(c.rank) * BM;
       const int n0 = nt * TILE_N;
@@ -1345,6 +1347,14 @@ tp_status grouped_gemm(const GemmArgs& g, cudaStream_t s) {
   if (tiles > INT32_MAX) return fail(TP_ESHAPE, "too many tiles");
   p.num_tiles = static_cast<int>(tiles);
   p.num_kb = static_cast<int>((g.K + BK - 1) / BK);
+  // Raster band: as many row-tiles as keep about RASTER_A_BYTES of A rows, so that the band's A stays in
+  // L2 while its B panels stream past. Measured on the sharded-matmul cases (K = 8192, 256-row tiles):
+  // 8 row-tiles instead of 16 read 0.4-0.9 GB less from DRAM per launch and ran 1-4% faster.
+  {
+    const int64_t a_tile = static_cast<int64_t>(pair ? 2 * BM : BM) * g.K * 2;
+    const int64_t fit = RASTER_A_BYTES / a_tile;
+    p.band = static_cast<int>(fit < 1 ? 1 : fit > RASTER_BAND_MAX ? RASTER_BAND_MAX : fit);
+  }
   p.status = status_word();
   p.budget = wait_budget();
   if (p.status == nullptr) return fail(TP_ECUDA, "cannot resolve the device status word");
