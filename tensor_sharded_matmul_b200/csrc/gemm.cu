@@ -35,7 +35,9 @@
 //     barriers count both CTAs' TMA bytes;
 //   * two TMEM accumulators of 256 columns, so the epilogue of one unit overlaps the main loop of the
 //     next;
-//   * the remaining warps: epilogue (tcgen05.ld 32 columns at a time);
+//   * the remaining warps: epilogue (tcgen05.ld 32 columns at a time; the plain GEMMs stage each
+//     warp's 32 x 32 output block through shared memory so that every store instruction writes
+//     whole row segments of 64 or 128 bytes);
 //   * every mbarrier wait is bounded: on expiry the kernel records the site in the status word,
 //     raises a shared abort flag, drains its in-flight copies and MMAs and frees TMEM.
 // No TMA load uses cluster multicast; the pair's commits reach both CTAs through tcgen05.commit's
@@ -308,6 +310,23 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
          (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(hi))) << 16);
 }
 
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, float a, float b, float c, float d) {
+  asm volatile("st.shared.v4.f32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
+}
+__device__ __forceinline__ void st_shared_u4(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+}
+__device__ __forceinline__ uint4 ld_shared_u4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ float4 ld_shared_v4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr) : "memory");
+  return v;
+}
+
 // ------------------------------------------------------------------ grouped GEMM
 struct GemmParams {
   CUtensorMap ta[TP_MAX_SHARDS];    // A views
@@ -347,31 +366,68 @@ __device__ __forceinline__ const CUtensorMap* a_view(const GemmParams& p, int g,
   return &p.ta[g];
 }
 
-// Store 32 consecutive output columns [col0, col0+32) of one row.
+
+// fp32 output of one warp: a 32 x 32 block held one row per lane (lane i: row row0 + i, columns col0..
+// col0+31), written through the warp's 4 KiB staging buffer. Its 16-byte pieces are XOR-swizzled by
+// row, so that the row-wise writes and the column-wise reads are free of bank conflicts, and each
+// store instruction covers four rows x 128 contiguous bytes instead of 32 rows x 16 bytes.
+__device__ __forceinline__ void store_f32_staged(void* cbase, int M, int N, uint32_t stg, int lane,
+                                                 const uint32_t (&v)[32], int row0, int col0) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    st_shared_v4(stg + lane * 128 + ((j ^ (lane & 7)) << 4), __uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                 __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+  __syncwarp();
+  const int sub = lane & 7;
+  float* c = static_cast<float*>(cbase);
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int r = 4 * k + (lane >> 3);
+    const float4 x = ld_shared_v4(stg + r * 128 + ((sub ^ (r & 7)) << 4));
+    const int row = row0 + r;
+    const int col = col0 + 4 * sub;   // N % 8 == 0: a vector inside N lies wholly inside it
+    if (row < M && col < N)
+      st_v4(c + static_cast<int64_t>(row) * N + col,
+            make_uint4(__float_as_uint(x.x), __float_as_uint(x.y), __float_as_uint(x.z), __float_as_uint(x.w)));
+  }
+  __syncwarp();
+}
+
+// bf16 output of one warp: 32 rows x 32 columns (64 bytes a row), one row per lane, formed by the
+// epilogue in registers (f: 32 values of this lane's row). Staged like store_f32_staged, with the
+// 64-byte swizzle (piece j of row r at piece j ^ ((r / 2) % 4)); each store instruction then covers
+// eight rows x 64 contiguous bytes.
+__device__ __forceinline__ void store_bf16_staged(void* cbase, int M, int N, uint32_t stg, int lane, const float (&f)[32],
+                                                  int row0, int col0) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    st_shared_u4(stg + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4),
+                 make_uint4(pack2(f[8 * j], f[8 * j + 1]), pack2(f[8 * j + 2], f[8 * j + 3]),
+                            pack2(f[8 * j + 4], f[8 * j + 5]), pack2(f[8 * j + 6], f[8 * j + 7])));
+  __syncwarp();
+  const int q = lane & 3;
+  uint16_t* c = static_cast<uint16_t*>(cbase);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int r = 8 * k + (lane >> 2);
+    const uint4 x = ld_shared_u4(stg + r * 64 + ((q ^ ((r >> 1) & 3)) << 4));
+    const int row = row0 + r;
+    const int col = col0 + 8 * q;   // N % 8 == 0: a vector inside N lies wholly inside it
+    if (row < M && col < N) st_v4(c + static_cast<int64_t>(row) * N + col, x);
+  }
+  __syncwarp();
+}
+
+// Applies the epilogue's activation to 32 accumulator columns (u: SwiGLU's up half).
 template <int EPI>
-__device__ __forceinline__ void store_row_chunk(void* cbase, int N, int row, int col0, const uint32_t (&v)[32],
-                                                const uint32_t (&u)[32]) {
-  if constexpr (EPI == EPI_F32) {
-    float* dst = static_cast<float*>(cbase) + static_cast<int64_t>(row) * N + col0;
+__device__ __forceinline__ void activate32(const uint32_t (&v)[32], const uint32_t (&u)[32], float (&f)[32]) {
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
-      if (col0 + 4 * j < N) st_v4(dst + 4 * j, make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
-  } else {
-    float f[32];
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const float x = __uint_as_float(v[j]);
-      if constexpr (EPI == EPI_BF16) f[j] = x;
-      else if constexpr (EPI == EPI_GELU) f[j] = gelu_erf(x);
-      else if constexpr (EPI == EPI_GELU_TANH) f[j] = gelu_tanh(x);
-      else f[j] = silu(x) * __uint_as_float(u[j]);
-    }
-    uint16_t* dst = static_cast<uint16_t*>(cbase) + static_cast<int64_t>(row) * N + col0;
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-      if (col0 + 8 * j < N)
-        st_v4(dst + 8 * j, make_uint4(pack2(f[8 * j], f[8 * j + 1]), pack2(f[8 * j + 2], f[8 * j + 3]),
-                                      pack2(f[8 * j + 4], f[8 * j + 5]), pack2(f[8 * j + 6], f[8 * j + 7])));
+  for (int j = 0; j < 32; ++j) {
+    const float x = __uint_as_float(v[j]);
+    if constexpr (EPI == EPI_BF16) f[j] = x;
+    else if constexpr (EPI == EPI_GELU) f[j] = gelu_erf(x);
+    else if constexpr (EPI == EPI_GELU_TANH) f[j] = gelu_tanh(x);
+    else f[j] = silu(x) * __uint_as_float(u[j]);
   }
 }
 
@@ -383,7 +439,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tcgen05_kernel(const __g
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint32_t* tmem_slot;
-  const Ctl c = setup_ctl(smem, 0, tmem_slot, p.status, p.budget, false, p.a_mn, p.b_km);
+  constexpr uint32_t STAGING = 4 * STAGING_PER_WARP;   // output staging, one buffer per epilogue warp
+  const Ctl c = setup_ctl(smem, STAGING, tmem_slot, p.status, p.budget, false, p.a_mn, p.b_km);
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
 
@@ -452,9 +509,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tcgen05_kernel(const __g
       const int n0 = nt * TILE_N;
       if (!wait_or_abort(c, c.accf0 + 8 * acc, acc_phase, WAIT_EPI_ACC_FULL)) break;
       tc_fence_after();
-      const int row = m0 + quad * 32 + lane;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * BN);
       void* cbase = p.c[g];
+      const uint32_t stg = smem_u32(smem + STAGES * (A_STAGE + B_STAGE)) + (warp - 2) * STAGING_PER_WARP;
 #pragma unroll 1
       for (int ch = 0; ch < TILE_N / 32; ++ch) {
         uint32_t v[32], u[32];
@@ -462,7 +519,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tcgen05_kernel(const __g
         if constexpr (SWIGLU) tmem_ld32(t_row + 128 + ch * 32, u);
         tmem_ld_wait();
         const int col0 = n0 + ch * 32;
-        if (row < p.M && col0 < p.N) store_row_chunk<EPI>(cbase, p.N, row, col0, v, u);
+        if constexpr (EPI == EPI_F32) {
+          store_f32_staged(cbase, p.M, p.N, stg, lane, v, m0 + quad * 32, col0);
+        } else {
+          float f[32];
+          activate32<EPI>(v, u, f);
+          store_bf16_staged(cbase, p.M, p.N, stg, lane, f, m0 + quad * 32, col0);
+        }
       }
       tc_fence_before();
       __syncwarp();
@@ -701,7 +764,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     for (int g = 0; g < p.n_amaps; ++g) prefetch_tmap(&p.ta[g]);
   }
   uint32_t* tmem_slot;
-  const PairCtl c = pair_setup(smem, 0, tmem_slot, 4, p.status, p.budget, false, p.a_mn, p.b_km);
+  constexpr uint32_t STAGING = 4 * STAGING_PER_WARP;   // output staging, one buffer per epilogue warp
+  const PairCtl c = pair_setup(smem, STAGING, tmem_slot, 4, p.status, p.budget, false, p.a_mn, p.b_km);
   const uint32_t tmem_base = *tmem_slot;
   const int pair = blockIdx.x >> 1;
   const int pairs = gridDim.x >> 1;
@@ -751,9 +815,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
       const int m0 = (rt - g * tiles_m) * TILE_M + static_cast<int>(c.rank) * BM;
       const int n0 = nt * TILE_N;
       if (!pair_wait_acc_full(c, acc, acc_phase)) break;
-      const int row = m0 + quad * 32 + lane;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(acc * BN);
       void* cbase = p.c[g];
+      const uint32_t stg = smem_u32(smem + PAIR_STAGES * (PAIR_A_STAGE + PAIR_B_STAGE)) + (warp - 2) * STAGING_PER_WARP;
 #pragma unroll 1
       for (int ch = 0; ch < TILE_N / 32; ++ch) {
         uint32_t v[32], u[32];
@@ -761,7 +825,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
         if constexpr (SWIGLU) tmem_ld32(t_row + 128 + ch * 32, u);
         tmem_ld_wait();
         const int col0 = n0 + ch * 32;
-        if (row < p.M && col0 < p.N) store_row_chunk<EPI>(cbase, p.N, row, col0, v, u);
+        if constexpr (EPI == EPI_F32) {
+          store_f32_staged(cbase, p.M, p.N, stg, lane, v, m0 + quad * 32, col0);
+        } else {
+          float f[32];
+          activate32<EPI>(v, u, f);
+          store_bf16_staged(cbase, p.M, p.N, stg, lane, f, m0 + quad * 32, col0);
+        }
       }
       pair_release_acc(c, acc, lane);
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
@@ -794,14 +864,6 @@ struct RingGemmParams {
   unsigned long long budget;
 };
 
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, float a, float b, float c, float d) {
-  asm volatile("st.shared.v4.f32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
-}
-__device__ __forceinline__ float4 ld_shared_v4(uint32_t addr) {
-  float4 v;
-  asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr) : "memory");
-  return v;
-}
 
 // Writes a 32 x 32 fp32 block held one row per lane (lane i: row row0+i, columns col0..col0+31)
 // with coalesced global stores. The block passes through the warp's 4 KiB staging buffer, with its
@@ -1197,22 +1259,24 @@ tp_status reserve_smem(K kernel, size_t bytes, int* done_for) {
 template <int EPI>
 tp_status launch(GemmParams& p, cudaStream_t s) {
   static int configured_for[64] = {};
-  if (tp_status st = reserve_smem(gemm_tcgen05_kernel<EPI>, GEMM_SMEM, configured_for)) return st;
+  constexpr size_t smem = GEMM_SMEM + 4 * STAGING_PER_WARP;
+  if (tp_status st = reserve_smem(gemm_tcgen05_kernel<EPI>, smem, configured_for)) return st;
   const int sms = sm_count();
   const int grid = p.num_tiles < sms ? p.num_tiles : sms;
-  gemm_tcgen05_kernel<EPI><<<grid, GEMM_THREADS, GEMM_SMEM, s>>>(p);
+  gemm_tcgen05_kernel<EPI><<<grid, GEMM_THREADS, smem, s>>>(p);
   return check_launch("gemm_tcgen05_kernel");
 }
 
 template <int EPI>
 tp_status launch_pair(GemmParams& p, cudaStream_t s) {
   static int configured_for[64] = {};
-  if (tp_status st = reserve_smem(gemm_pair_kernel<EPI>, PAIR_SMEM, configured_for)) return st;
+  constexpr size_t smem = PAIR_SMEM + 4 * STAGING_PER_WARP;
+  if (tp_status st = reserve_smem(gemm_pair_kernel<EPI>, smem, configured_for)) return st;
   const int sms = sm_count();
   const int tiles = p.groups * ((p.M + 2 * BM - 1) / (2 * BM)) * p.tiles_n;
   int grid = 2 * tiles < sms ? 2 * tiles : (sms & ~1);
   if (grid < 2) grid = 2;
-  gemm_pair_kernel<EPI><<<grid, GEMM_THREADS, PAIR_SMEM, s>>>(p);
+  gemm_pair_kernel<EPI><<<grid, GEMM_THREADS, smem, s>>>(p);
   return check_launch("gemm_pair_kernel");
 }
 
