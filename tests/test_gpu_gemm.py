@@ -57,7 +57,8 @@ def test_gemm_fp32_out(groups, M, N, K, shared):
 
 @pytest.mark.parametrize("act", ["none", "gelu", "gelu_tanh"])
 @pytest.mark.parametrize("groups,M,N,K", [(2, 256, 512, 512), (4, 64, 256, 256), (3, 200, 136, 96),
-                                          (2, 1024, 2560, 256)])   # more tiles than CTA pairs
+                                          (2, 1024, 2560, 256),    # more tiles than CTA pairs
+                                          (2, 384, 264, 128)])     # CTA pairs: a half-empty row tile, 8-column tail
 def test_gemm_bf16_epilogues(act, groups, M, N, K):
     got, ref = _run(groups, M, N, K, act, tp.TP_BF16, shared_a=True, seed=N)
     for g in range(groups):
