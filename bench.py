@@ -771,9 +771,13 @@ def run_cases(args) -> int:
         c, st = (int(v) for v in args.case.split("."))
         which = {(c, st)}
     iters = args.steps if args.steps < 500 else None
+    import tensor_sharded_matmul_b200 as tp
     for case_id, strategy, name, ms, rate, nbytes in sharded_matmul_cases(which, iters):
+        # the strategy the pages' byte rule would pick on t devices (case 3: the output sharding decides)
+        rule = tp.tp_sharded_matmul_choose(case_id, 8192, 8192, 28672, 4) if case_id != 3 else None
         _emit({"config": "sharded_matmul", "case": case_id, "strategy": name, "ms": ms, "tflops_executed": rate,
-               "frac_bf16_peak": rate / peak, "workspace_bytes": nbytes})
+               "frac_bf16_peak": rate / peak, "workspace_bytes": nbytes,
+               "cost_rule_choice": None if rule is None else rule == strategy})
     return 0
 
 

@@ -279,6 +279,19 @@ tp_status tp_mlp_fwd_sp(const uint16_t* const* x, int64_t N, int64_t h, int64_t 
  *     (each 128-row tile of X likewise), case 4 GATHER_W with (F/t) % 64 == 0 (each 64-column box
  *     of W likewise). Otherwise the gather is materialised in the workspace, one copy per shard. */
 size_t tp_sharded_matmul_ws_bytes(int case_id, int strategy, int64_t B, int64_t D, int64_t F, int t);
+/* The strategy that the pages' cost rule picks ([CH06] §6.2 cases 2 and 4, §6.9 Problem 4), written
+ * to *strategy. The rule compares the elements a ring of t devices would move, taking operands and
+ * output to have the same element type:
+ *   case 1  TP_CASE1_LOCAL: nothing moves;
+ *   case 2  TP_CASE2_ALLGATHER when gathering X (B*D elements) moves no more than the AllReduce of
+ *           C (about 2*B*F), else TP_CASE2_ALLREDUCE. For the weight-gathering orientation of
+ *           Problem 4 this is the page's "AllReduce when D > 2B";
+ *   case 4  gather the smaller operand: TP_CASE4_GATHER_X when B*D <= D*F, else TP_CASE4_GATHER_W;
+ *   case 3  TP_EUNSUPPORTED: its three strategies reduce the same partials, and the sharding the
+ *           caller wants for C decides among them (replicated, rows or columns).
+ * On one GPU the gathers cost no traffic (the GEMM reads the pieces in place); this reports the
+ * multi-device choice. Host-only; sizes must be positive, 1 <= t <= TP_MAX_SHARDS (TP_EINVAL). */
+tp_status tp_sharded_matmul_choose(int case_id, int64_t B, int64_t D, int64_t F, int t, int* strategy);
 tp_status tp_sharded_matmul(int case_id, int strategy, const uint16_t* const* x, const uint16_t* const* w,
                             int64_t B, int64_t D, int64_t F, int t, void* const* c, tp_dtype c_dtype,
                             void* ws, size_t ws_bytes, void* stream);

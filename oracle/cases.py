@@ -113,6 +113,13 @@ def to_logical(outs, layout: str):
     raise ValueError(layout)
 
 
+def case4_choice(B: int, D: int, F: int) -> str:
+    """Case 4 fixes the doubly-sharded contraction by gathering one operand; the page leaves which one
+    open ("Scaling Book 入门第 6 章", §6.2 Case 4: it depends). Reading: gather the smaller one, as the
+    byte count of an AllGather is the operand's size. X[B_X, D] has B*D elements, W[D, F_X] D*F."""
+    return "gather_x" if B * D <= D * F else "gather_w"
+
+
 def case2_choice(gathered_elems: int, output_elems: int) -> str:
     """Pick the case-2 strategy by bytes moved (ring, bandwidth-bound, same dtype): AllGather of the
     operand sharded on the contracting dim moves about its full size; AllReduce of the output about

@@ -35,7 +35,7 @@ EXPORTED = (
     "tp_status_str", "tp_last_error", "tp_device_status", "tp_set_wait_budget", "tp_selftest_wait_timeout",
     "tp_num_sms", "tp_shard_cols", "tp_shard_rows", "tp_shard_gate_up", "tp_shard_qkv", "tp_reduce_scatter",
     "tp_all_gather", "tp_all_reduce", "tp_grouped_gemm", "tp_column_linear", "tp_row_linear", "tp_row_linear_reduce", "tp_mlp_fwd",
-    "tp_sharded_matmul_ws_bytes", "tp_sharded_matmul", "tp_layer_fwd", "tp_mlp_fwd_noalloc",
+    "tp_sharded_matmul_ws_bytes", "tp_sharded_matmul_choose", "tp_sharded_matmul", "tp_layer_fwd", "tp_mlp_fwd_noalloc",
     "tp_column_linear_sp", "tp_mlp_fwd_sp", "tp_all_to_all", "tp_grouped_gemm_t", "tp_mlp_bwd",
 )
 
@@ -68,6 +68,7 @@ _SIGS = {
     "tp_column_linear_sp": (_i32, [_pp, _i64, _i64, _i64, _i32, _i32, _vp, _vp, _vp]),
     "tp_mlp_fwd_sp": (_i32, [_pp, _i64, _i64, _i64, _i32, _i32, _vp, _vp, _vp, _pp, _vp]),
     "tp_sharded_matmul_ws_bytes": (_sz, [_i32, _i32, _i64, _i64, _i64, _i32]),
+    "tp_sharded_matmul_choose": (_i32, [_i32, _i64, _i64, _i64, _i32, C.POINTER(C.c_int)]),
     "tp_sharded_matmul": (_i32, [_i32, _i32, _pp, _pp, _i64, _i64, _i64, _i32, _pp, _i32, _vp, _sz, _vp]),
     "tp_layer_fwd": (_i32, [_vp, _pp, _i64, _i64, _i32, _i32, _i32, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _pp,
                             _vp, _vp, _pp, _pp, _vp]),
@@ -233,6 +234,13 @@ def tp_mlp_fwd_sp(x, N, h, F, t, act, w_in, w_down, z_ws, out, stream=None):
 
 def tp_sharded_matmul_ws_bytes(case_id, strategy, B, D, F, t) -> int:
     return int(_lib.tp_sharded_matmul_ws_bytes(case_id, strategy, B, D, F, t))
+
+
+def tp_sharded_matmul_choose(case_id, B, D, F, t) -> int:
+    """The strategy the pages' cost rule picks for case 1, 2 or 4 (see include/tp.h)."""
+    out = C.c_int(-1)
+    _call("tp_sharded_matmul_choose", case_id, B, D, F, t, C.byref(out))
+    return out.value
 
 
 def tp_sharded_matmul(case_id, strategy, x, w, B, D, F, t, c, c_dtype, ws, ws_bytes, stream=None):

@@ -269,6 +269,23 @@ size_t tp_sharded_matmul_ws_bytes(int case_id, int strategy, int64_t B, int64_t 
   }
 }
 
+tp_status tp_sharded_matmul_choose(int case_id, int64_t B, int64_t D, int64_t F, int t, int* strategy) {
+  if (strategy == nullptr) return fail(TP_EINVAL, "null strategy pointer");
+  if (!valid_t(t)) return fail(TP_EINVAL, "t=%d outside 1..%d", t, TP_MAX_SHARDS);
+  if (B <= 0 || D <= 0 || F <= 0) return fail(TP_EINVAL, "sizes must be positive");
+  switch (case_id) {
+    case 1: *strategy = TP_CASE1_LOCAL; return TP_OK;
+    case 2: {   // gathered X: B*D elements; AllReduce of C: about 2*B*F (both in 128-bit arithmetic)
+      const __int128 gathered = static_cast<__int128>(B) * D, reduced = static_cast<__int128>(2) * B * F;
+      *strategy = gathered <= reduced ? TP_CASE2_ALLGATHER : TP_CASE2_ALLREDUCE;
+      return TP_OK;
+    }
+    case 3: return fail(TP_EUNSUPPORTED, "case 3: the wanted sharding of C picks AllReduce, RS_B or RS_F");
+    case 4: *strategy = B <= F ? TP_CASE4_GATHER_X : TP_CASE4_GATHER_W; return TP_OK;   // B*D <= D*F
+    default: return fail(TP_EINVAL, "case %d outside 1..4", case_id);
+  }
+}
+
 tp_status tp_sharded_matmul(int case_id, int strategy, const uint16_t* const* x, const uint16_t* const* w, int64_t B,
                             int64_t D, int64_t F, int t, void* const* c, tp_dtype c_dtype, void* ws, size_t ws_bytes,
                             void* stream) {

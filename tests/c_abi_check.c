@@ -34,5 +34,14 @@ int main(void) {
   printf("ws_case4_gather_w %zu\n", tp_sharded_matmul_ws_bytes(4, TP_CASE4_GATHER_W, 8192, 8192, 28672, 4));
   printf("ws_case4_gather_w_ragged %zu\n", tp_sharded_matmul_ws_bytes(4, TP_CASE4_GATHER_W, 8192, 8192, 384, 4));
   printf("ws_case3_fused %zu\n", tp_sharded_matmul_ws_bytes(3, TP_CASE3_RS_B, 8192, 8192, 28672, 4));
+  /* strategy choice by the pages' byte rule (host arithmetic) */
+  {
+    int st2 = -1, st4 = -1;
+    tp_status a = tp_sharded_matmul_choose(2, 8192, 8192, 28672, 4, &st2);
+    tp_status b = tp_sharded_matmul_choose(4, 8192, 8192, 28672, 4, &st4);
+    printf("choose_case2 %d %d\n", (int)a, st2);
+    printf("choose_case4 %d %d\n", (int)b, st4);
+    printf("choose_case3 %d\n", (int)tp_sharded_matmul_choose(3, 8192, 8192, 28672, 4, &st2));
+  }
   return 0;
 }

@@ -189,3 +189,33 @@ def test_per_hop_bf16_is_a_ring_collective_mode_only():
     # empty inputs pass validation in the per-hop mode like in the others
     tp.tp_reduce_scatter([0, 0], [0, 0], 0, 16, 0, tp.TP_BF16_RING, 2, 0)
     tp.tp_all_reduce([0, 0], [0, 0], 0, 16, tp.TP_BF16_RING, 2, 0)
+
+
+def test_strategy_choice_matches_the_oracle_rule():
+    """tp_sharded_matmul_choose applies the pages' byte rule (case 2: AllGather of X unless it moves
+    more than the AllReduce of C; case 4: gather the smaller operand) like oracle.cases does."""
+    from oracle import cases as OC
+    code2 = {"allgather": tp.TP_CASE2_ALLGATHER, "allreduce": tp.TP_CASE2_ALLREDUCE}
+    code4 = {"gather_x": tp.TP_CASE4_GATHER_X, "gather_w": tp.TP_CASE4_GATHER_W}
+    shapes = [(8192, 8192, 28672), (4096, 4096, 14336), (64, 256, 1024)]
+    for B in (8, 256, 4096):
+        for F in (B // 2, B, 2 * B):
+            for D in (2 * F - 8, 2 * F, 2 * F + 8):   # around the case-2 boundary B*D = 2*B*F
+                if D > 0:
+                    shapes.append((B, D, F))
+    shapes += [(B, 512, B + d) for B in (16, 1024) for d in (-8, 0, 8)]   # around the case-4 boundary
+    for B, D, F in shapes:
+        assert tp.tp_sharded_matmul_choose(1, B, D, F, 4) == tp.TP_CASE1_LOCAL
+        assert tp.tp_sharded_matmul_choose(2, B, D, F, 4) == code2[OC.case2_choice(B * D, B * F)], (B, D, F)
+        assert tp.tp_sharded_matmul_choose(4, B, D, F, 4) == code4[OC.case4_choice(B, D, F)], (B, D, F)
+    # the benchmark's configuration: gather X for both cases
+    assert tp.tp_sharded_matmul_choose(2, 8192, 8192, 28672, 4) == tp.TP_CASE2_ALLGATHER
+    assert tp.tp_sharded_matmul_choose(4, 8192, 8192, 28672, 4) == tp.TP_CASE4_GATHER_X
+    # huge sizes do not overflow the comparison
+    assert tp.tp_sharded_matmul_choose(2, 1 << 40, 1 << 41, 1 << 40, 4) == tp.TP_CASE2_ALLGATHER
+    assert tp.tp_sharded_matmul_choose(2, 1 << 40, (1 << 41) + 8, 1 << 40, 4) == tp.TP_CASE2_ALLREDUCE
+    _expect(tp.TP_EUNSUPPORTED, tp.tp_sharded_matmul_choose, 3, 8192, 8192, 28672, 4)
+    _expect(tp.TP_EINVAL, tp.tp_sharded_matmul_choose, 5, 8192, 8192, 28672, 4)
+    _expect(tp.TP_EINVAL, tp.tp_sharded_matmul_choose, 2, 0, 8192, 28672, 4)
+    _expect(tp.TP_EINVAL, tp.tp_sharded_matmul_choose, 2, 8192, 8192, 28672, 17)
+

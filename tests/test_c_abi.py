@@ -46,3 +46,6 @@ def test_workspace_sizes_from_c(c_output):
     assert int(c_output["ws_case4_gather_w"]) == 0                 # W's pieces read in place
     assert int(c_output["ws_case4_gather_w_ragged"]) == 4 * 8192 * 384 * 2   # F/t = 96: gathered copy
     assert int(c_output["ws_case3_fused"]) == 0
+    assert c_output["choose_case2"] == f"{tp.TP_OK} {tp.TP_CASE2_ALLGATHER}"
+    assert c_output["choose_case4"] == f"{tp.TP_OK} {tp.TP_CASE4_GATHER_X}"
+    assert int(c_output["choose_case3"]) == tp.TP_EUNSUPPORTED
