@@ -48,6 +48,10 @@ def _run(groups, M, N, K, act, c_dtype, shared_a, seed=0):
     # CTA pairs take two k-blocks per pipeline stage: odd k-block counts leave the last stage half used
     (2, 256, 256, 64, False),     # one k-block
     (1, 512, 512, 136, True),     # three k-blocks, the last ragged
+    # long contractions shrink the raster band (row-tiles kept in L2 together): 8 row-tiles at
+    # K = 8192 (12 here: one full band and a partial one), 4 at K = 16384
+    (3, 1024, 512, 8192, False),
+    (2, 1280, 264, 16384, True),
 ])
 def test_gemm_fp32_out(groups, M, N, K, shared):
     got, ref = _run(groups, M, N, K, "none", tp.TP_F32, shared, seed=M + N + K)
