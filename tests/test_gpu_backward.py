@@ -82,3 +82,63 @@ def test_mlp_backward_against_oracle(N, h, F, t, act):
         assert_close(f64(g_in[r]), ref["dW_in"][r], GEMM_TOL, f"dW_in[{r}]")
         assert_close(f64(gx[r]), ref["dX"], GEMM_TOL, f"dX replica {r}")
         assert same_bits(host_bits(gx[r]), host_bits(gx[0]))   # f's backward AllReduce: identical replicas
+
+
+def _sample(n: int, tile: int = 128) -> np.ndarray:
+    """One index from every `tile`-wide block (at an offset that moves from block to block, so that
+    different TMEM lanes, epilogue warps and both CTAs of a pair are checked), plus the first and
+    the last index."""
+    idx = {0, n - 1}
+    for b in range(n // tile):
+        idx.add(b * tile + (b * 53 + 17) % tile)
+    return np.array(sorted(idx))
+
+
+def test_llama8b_backward_full_size_sampled():
+    """The backward at the benchmark's Llama-3-8B shape (4096 tokens, h = 4096, F = 14336, t = 8,
+    SwiGLU) against the oracle, on samples the oracle computes exactly:
+      * dX and dH on one row per 128-row tile: a row of either needs only the same row of X and dY,
+        so the oracle runs on those rows alone;
+      * dW_down rows and dW_in columns on one index per 128-wide block of F/t, for three shards: those
+        slices need only the matching gate/up columns of W_in and rows of W_down, so the oracle runs
+        on the sliced shards with the full X and dY."""
+    from oracle import layouts as OL
+    N, h, F, t = 4096, 4096, 14336, 8
+    f = F // t
+    X, Wgu, Wd = S.llama8b_mlp(seed=0)
+    dY = S.Draw(7).normal((N, h), 1.0)
+    dX_, ddY = cuda(X), cuda(dY)
+    dWgu, dWd = cuda(Wgu), cuda(Wd)
+    w_in = torch.empty((t, h, 2 * f), dtype=torch.bfloat16, device="cuda")
+    w_down = torch.empty((t, f, h), dtype=torch.bfloat16, device="cuda")
+    tp.tp_shard_gate_up(dWgu, 2 * F, dWgu.data_ptr() + 2 * F, 2 * F, h, F, t, w_in)
+    tp.tp_shard_rows(dWd, h, F, h, t, w_down)
+    del dWgu, dWd
+    H, Z = _forward_intermediates(dX_, w_in, N, h, F, t, "swiglu")
+    dz = torch.empty((t, N, f), dtype=torch.bfloat16, device="cuda")
+    dh = torch.empty((t, N, 2 * f), dtype=torch.bfloat16, device="cuda")
+    g_in = torch.empty((t, h, 2 * f), device="cuda")
+    g_down = torch.empty((t, f, h), device="cuda")
+    gx = [torch.empty((N, h), device="cuda") for _ in range(t)]
+    tp.tp_mlp_bwd(dX_, ddY, N, h, F, t, tp.TP_ACT_SWIGLU, w_in, w_down, H, Z, dz, dh, g_in, g_down, gx)
+    torch.cuda.synchronize()
+    st, site = tp.tp_device_status(1)
+    assert st == tp.TP_OK, f"device wait site {site}"
+    shards_in = list(OL.shard_gate_up(Wgu[:, :F].float().numpy(), Wgu[:, F:].float().numpy(), t))
+    shards_down = list(OL.shard_rows(Wd.float().numpy(), t))
+    Xf, dYf = f64(X), f64(dY)
+
+    rows = _sample(N)
+    ref = OM.mlp_backward(Xf[rows], shards_in, shards_down, dYf[rows], "swiglu")
+    for r in (0, 3, 7):
+        assert_close(f64(gx[r])[rows], ref["dX"], GEMM_TOL, f"dX replica {r}")
+        assert_close(f64(dh[r])[rows], ref["dH"][r], GEMM_TOL, f"dH[{r}]")
+    for r in range(t):
+        assert same_bits(host_bits(gx[r]), host_bits(gx[0]))   # the AllReduce's replicas are identical
+
+    cols = _sample(f)
+    gate_up = np.concatenate([cols, f + cols])
+    for s in (0, 3, 7):
+        sub = OM.mlp_backward(Xf, [shards_in[s][:, gate_up]], [shards_down[s][cols, :]], dYf, "swiglu")
+        assert_close(f64(g_down[s])[cols, :], sub["dW_out"][0], GEMM_TOL, f"dW_down[{s}] rows")
+        assert_close(f64(g_in[s])[:, gate_up], sub["dW_in"][0], GEMM_TOL, f"dW_in[{s}] columns")
