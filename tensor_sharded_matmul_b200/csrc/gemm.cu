@@ -20,9 +20,9 @@
 //    registers, one binary32 add per shard, which is exactly the ReduceScatter's summation order. It
 //    then writes the tile once: to shard c's output (ReduceScatter) or to all t outputs (AllReduce =
 //    ReduceScatter followed by AllGather, its chunks rows or columns), optionally adding a residual
-//    and writing a bf16 copy. The
-//    fp32 partials never reach HBM. Each U_s tile comes from the same MMA instruction sequence as the
-//    plain GEMM's, so the results are bit-identical to the unfused GEMM followed by the ring kernel.
+//    and writing a bf16 copy. The fp32 partials never reach HBM. Each U_s tile comes from the same
+//    MMA instruction sequence as the plain GEMM's, so the results are bit-identical to the unfused
+//    GEMM followed by the ring kernel.
 //
 // Pipeline (sm_100a):
 //   * warp 0, one lane: TMA producer. A [M,K] is K-major (64 x 128 boxes, 128-byte swizzle); B [K,N]
@@ -35,6 +35,8 @@
 //     barriers count both CTAs' TMA bytes;
 //   * two TMEM accumulators of 256 columns, so the epilogue of one unit overlaps the main loop of the
 //     next;
+//   * tiles in raster bands of row-tiles swept across the n-tiles, each band holding about 32 MiB
+//     of A rows so that they stay in L2 while the band's B panels stream past;
 //   * the remaining warps: epilogue (tcgen05.ld 32 columns at a time; the plain GEMMs stage each
 //     warp's 32 x 32 output block through shared memory so that every store instruction writes
 //     whole row segments of 64 or 128 bytes);
